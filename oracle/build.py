@@ -1,0 +1,30 @@
+"""Compile the float64 oracle (plain C) into oracle/liblq_oracle.so.
+
+Test infrastructure: the oracle library is built here so tests, the smoke
+check and the benchmark's CPU-baseline leg can load it; the CUDA library
+never links or loads it.
+"""
+
+from __future__ import annotations
+
+import os
+import subprocess
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "lq_oracle.c")
+LIB = os.path.join(HERE, "liblq_oracle.so")
+
+
+def build(force: bool = False) -> str:
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+        return LIB
+    tmp = LIB + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-Wall", "-Wextra",
+           "-o", tmp, SRC]
+    subprocess.check_call(cmd)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force=True))
