@@ -1,0 +1,522 @@
+"""Benchmark of the LiftQuant lift-then-project layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lq|reference]
+
+Workload at N=1: the LQ-24/10 decode layer (in=5120, out=13824, lifted K=12288,
+batch 1, 40 orthogonal 128x128 whitening blocks, bf16 activations). One step is
+one pass of the decode hot path over one batch: whitening + lift
+(lq_lift_activations) then the 1-bit GEMV with the row-scale epilogue
+(lq_gemv). The metric is packed-weight GB/s: packed sign bytes (out*K/8) per
+step divided by the step time.
+
+Timing: weights (packed signs, s, T^-1) rotate over enough distinct copies to
+exceed 3x the L2 size, so every step reads its weights from HBM. Steps are
+replayed from CUDA graphs (16 steps per graph, one per weight copy) so that
+host launch overhead does not pace the GPU; the timed region is bracketed by a
+barrier and device synchronizes and timed with CUDA events on the launching
+stream; the reported time is the max over ranks. With N>1 every rank runs an
+independent replica (the layer needs no exchange between GPUs), so scaling is
+weak and the value sums all ranks' bytes over the slowest rank's time.
+
+One JSON line is printed by rank 0; it carries the roofline of the dominant
+kernel (the GEMV, timed alone right after the step region), the end-to-end
+number (pinned-host activations in, output back to the host, inside the timed
+region), sampled SM clocks, the float64 oracle timed on the host cores, and
+secondary results (prefill GEMM TFLOP/s, the LQ-20/8 batch sweep, the LQ-D/8
+bit-width sweep).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from datagen import CONFIGS, make_layer  # noqa: E402
+
+STEPS_PER_GRAPH = 16
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profiled_traffic(kernel_key):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/ (None if absent)."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        with open(path) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 2 and parts[0] == kernel_key:
+                    return float(parts[1])
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._reader = threading.Thread(target=self._read, daemon=True)
+            self._reader.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        if which == "begin":
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            rows.append((ts, parts))
+        if not rows:
+            return None
+        inside = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= (self.t1 or r[0])]
+        use = inside if inside else rows
+        sm = [float(p[1]) for _, p in use if p[1].replace(".", "").isdigit()]
+        smax = max(float(p[2]) for _, p in use if p[2].replace(".", "").isdigit())
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for _, p in use:
+            for n, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x, world, device=None):
+    """Max of a float over all ranks (identity when world == 1)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------------ GPU workloads
+
+class DecodeLayer:
+    """Device buffers of one decode workload, rotated over `copies` weight copies."""
+
+    def __init__(self, lq, cfg, batch, copies, torch):
+        L = make_layer(cfg, batch)
+        self.cfg, self.batch = cfg, batch
+        dev = torch.device("cuda")
+        pk = torch.from_numpy(L.packed.view(np.int32)).to(dev)
+        s = torch.from_numpy(L.s).to(dev)
+        tinv = torch.from_numpy(L.tinv).to(dev) if L.tinv is not None else None
+        self.packed = [pk] + [pk.clone() for _ in range(copies - 1)]
+        self.s = [s] + [s.clone() for _ in range(copies - 1)]
+        self.tinv = [tinv] + [tinv.clone() if tinv is not None else None for _ in range(copies - 1)]
+        self.M = torch.from_numpy(L.M).to(dev)
+        if L.a_dtype == "bf16":
+            a = torch.from_numpy(L.a.view(np.int16)).to(dev).view(torch.bfloat16)
+        else:
+            a = torch.from_numpy(L.a).to(dev)
+        self.a = [a.clone() for _ in range(copies)]
+        self.a_host = [x.cpu().pin_memory() for x in self.a]
+        self.u = [torch.empty((batch, cfg.K), dtype=torch.float32, device=dev) for _ in range(copies)]
+        self.o = [torch.empty((batch, cfg.out), dtype=torch.float32, device=dev) for _ in range(copies)]
+        self.o_host = [torch.empty((batch, cfg.out), dtype=torch.float32).pin_memory() for _ in range(copies)]
+        self.copies = copies
+        self.lq = lq
+
+    def step(self, i, with_copies=False):
+        lq, c = self.lq, self.cfg
+        if with_copies:
+            self.a[i].copy_(self.a_host[i], non_blocking=True)
+        lq.lift_activations(self.a[i], self.M, c.K, tinv=self.tinv[i], out=self.u[i])
+        lq.gemv(self.packed[i], self.s[i], self.u[i], out=self.o[i])
+        if with_copies:
+            self.o_host[i].copy_(self.o[i], non_blocking=True)
+
+    def gemv_only(self, i):
+        self.lq.gemv(self.packed[i], self.s[i], self.u[i], out=self.o[i])
+
+    @property
+    def packed_bytes(self):
+        return self.cfg.out * self.cfg.K // 8
+
+
+def copies_for(bytes_per_copy, l2_bytes):
+    return max(STEPS_PER_GRAPH, int(np.ceil(3 * l2_bytes / bytes_per_copy)))
+
+
+def capture(torch, fn, n):
+    """CUDA graph of fn(0..n-1) on a side stream (each fn launches through the C ABI)."""
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(n):   # warm-up outside capture (sets kernel attributes once)
+            fn(i)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            fn(i)
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(torch, graph, reps, per_rep):
+    """ms per unit: `reps` replays, each doing `per_rep` units, timed with events."""
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(st)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / (reps * per_rep)
+
+
+def run_steps(torch, graph_full, graphs_single, steps):
+    """Replay exactly `steps` steps: full 16-step graphs, then single-step graphs."""
+    full, rem = divmod(steps, STEPS_PER_GRAPH)
+    for _ in range(full):
+        graph_full.replay()
+    for i in range(rem):
+        graphs_single[i].replay()
+
+
+# ------------------------------------------------------------------ oracle on host cores
+
+def oracle_sample(cfg_name, budget_s, nthreads):
+    """The float64 oracle on the host: whitening + lift + contraction of the decode
+    layer, on as many output rows as fit in `budget_s`. Returns (GB/s of packed
+    weights, description)."""
+    import oracle
+    cfg = CONFIGS[cfg_name]
+    L = make_layer(cfg, 1)
+    a = oracle.to_f64(L.a, L.a_dtype)
+    t = None if L.tinv is None else oracle.to_f64(L.tinv)
+    M = oracle.to_f64(L.M)
+    # calibrate on 64 rows
+    t0 = time.perf_counter()
+    u, _ = oracle.forward(L.packed[:64], L.s[:64], a, t, M, cfg.K, nthreads)
+    dt = time.perf_counter() - t0
+    rows = int(min(cfg.out, max(64, 64 * budget_s / max(dt, 1e-6))))
+    t0 = time.perf_counter()
+    oracle.forward(L.packed[:rows], L.s[:rows], a, t, M, cfg.K, nthreads)
+    dt = time.perf_counter() - t0
+    gbs = rows * cfg.K / 8 / dt / 1e9
+    return gbs, dt, f"{cfg_name}: whitening + lift + sign contraction of {rows} of {cfg.out} rows, batch 1"
+
+
+def reference_arm(args, world, rank):
+    """`--impl reference`: the float64 oracle on the host cores as the reference arm."""
+    if rank != 0:
+        return
+    import oracle
+    nthreads = oracle.threads_available()
+    total_budget = 90.0
+    per_step = total_budget / max(1, args.steps + args.warmup)
+    for _ in range(args.warmup):
+        oracle_sample(args.workload, per_step, nthreads)
+    vals, times = [], []
+    for _ in range(args.steps):
+        v, dt, desc = oracle_sample(args.workload, per_step, nthreads)
+        vals.append(v)
+        times.append(dt)
+    value = float(np.median(vals))
+    cfg = CONFIGS[args.workload]
+    line = {
+        "impl": "reference", "metric": "decode GEMV packed-weight GB/s", "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": float(np.median(times) * 1e3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "in": cfg.in_dim, "out": cfg.out, "d": cfg.d, "D": cfg.D,
+                   "K": cfg.K, "batch": 1},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": nthreads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main arm
+
+def bench_decode_sweep(torch, lq, name, batches, l2, reps=50):
+    cfg = CONFIGS[name]
+    res = {}
+    for b in batches:
+        probe = make_layer(cfg, b, packed=False)
+        per_copy = cfg.out * cfg.K // 8 + (probe.tinv.nbytes if probe.tinv is not None else 0)
+        layer = DecodeLayer(lq, cfg, b, copies_for(per_copy, l2), torch)
+        g = capture(torch, layer.step, STEPS_PER_GRAPH)
+        gg = capture(torch, layer.gemv_only, STEPS_PER_GRAPH)
+        for _ in range(3):
+            g.replay()
+        ms_step = time_graph(torch, g, reps, STEPS_PER_GRAPH)
+        ms_gemv = time_graph(torch, gg, reps, STEPS_PER_GRAPH)
+        res[str(b)] = {"step_us": ms_step * 1e3, "gemv_us": ms_gemv * 1e3,
+                       "gemv_GBps": layer.packed_bytes / (ms_gemv * 1e-3) / 1e9,
+                       "layer_tokens_per_s": b / (ms_step * 1e-3)}
+        del g, gg, layer
+        torch.cuda.empty_cache()
+    return res
+
+
+def bench_prefill(torch, lq, name, tokens, reps=10):
+    cfg = CONFIGS[name]
+    L = make_layer(cfg, tokens)
+    dev = torch.device("cuda")
+    pk = torch.from_numpy(L.packed.view(np.int32)).to(dev)
+    s = torch.from_numpy(L.s).to(dev)
+    tinv = torch.from_numpy(L.tinv).to(dev)
+    M = torch.from_numpy(L.M).to(dev)
+    a = torch.from_numpy(L.a.view(np.int16)).to(dev).view(torch.bfloat16)
+    u = torch.empty((tokens, cfg.K), dtype=torch.bfloat16, device=dev)
+    o = torch.empty((tokens, cfg.out), dtype=torch.float32, device=dev)
+    flush = torch.empty(int(400e6) // 4, dtype=torch.float32, device=dev)
+    st = torch.cuda.current_stream()
+
+    def t_of(fn):
+        for _ in range(3):
+            fn()
+        times = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            fn()
+            e1.record(st)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        return float(np.median(times))
+
+    ms_lift = t_of(lambda: lq.lift_activations(a, M, cfg.K, tinv=tinv, u_dtype="bf16", out=u))
+    ms_gemm = t_of(lambda: lq.gemm(pk, s, u, out=o))
+    flops = 2.0 * tokens * cfg.out * cfg.K
+    return {"tokens": tokens, "lift_us": ms_lift * 1e3, "gemm_us": ms_gemm * 1e3,
+            "gemm_TFLOPs": flops / (ms_gemm * 1e-3) / 1e12,
+            "layer_tokens_per_s": tokens / ((ms_lift + ms_gemm) * 1e-3)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=160000)
+    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--impl", default="lq", choices=["lq", "reference"])
+    ap.add_argument("--workload", default="decode_lq24_10")
+    ap.add_argument("--no-extra", action="store_true", help="skip the secondary sweeps")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_setup()
+
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        return
+
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    import bit_lifted_gemm_b200 as lq
+
+    peaks, peaks_src = load_peaks()
+    props = torch.cuda.get_device_properties(device)
+    l2 = getattr(props, "L2_cache_size", 126 * 2**20) or 126 * 2**20
+    cfg = CONFIGS[args.workload]
+    probe = make_layer(cfg, 1, packed=False)
+    per_copy = cfg.out * cfg.K // 8 + (probe.tinv.nbytes if probe.tinv is not None else 0) + 4 * cfg.out
+    copies = copies_for(per_copy, l2)
+    copies = (copies + STEPS_PER_GRAPH - 1) // STEPS_PER_GRAPH * STEPS_PER_GRAPH
+    layer = DecodeLayer(lq, cfg, 1, copies, torch)
+
+    # one graph per 16-step block of distinct weight copies
+    blocks = copies // STEPS_PER_GRAPH
+    g_full = [capture(torch, lambda i, b=b: layer.step(b * STEPS_PER_GRAPH + i), STEPS_PER_GRAPH)
+              for b in range(blocks)]
+    g_single = [capture(torch, lambda i, j=j: layer.step(j), 1) for j in range(STEPS_PER_GRAPH)]
+    g_gemv = [capture(torch, lambda i, b=b: layer.gemv_only(b * STEPS_PER_GRAPH + i), STEPS_PER_GRAPH)
+              for b in range(blocks)]
+    g_e2e = [capture(torch, lambda i, b=b: layer.step(b * STEPS_PER_GRAPH + i, with_copies=True), STEPS_PER_GRAPH)
+             for b in range(blocks)]
+
+    def replay_steps(graphs, n):
+        full, rem = divmod(n, STEPS_PER_GRAPH)
+        for k in range(full):
+            graphs[k % len(graphs)].replay()
+        for i in range(rem):
+            g_single[i].replay()
+
+    st = torch.cuda.current_stream()
+    replay_steps(g_full, args.warmup)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier(world, device)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.mark("begin")
+    e0.record(st)
+    replay_steps(g_full, args.steps)
+    e1.record(st)
+    e1.synchronize()
+    sampler.mark("end")
+    torch.cuda.synchronize()
+    barrier(world, device)
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, device)
+    clocks = sampler.stop()
+    ms_per_step = ms_total / args.steps
+    launches = 2 * args.steps
+
+    # dominant kernel alone (same stream, right after the step region)
+    reps = max(1, min(2000, args.steps // STEPS_PER_GRAPH))
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(st)
+    for k in range(reps):
+        g_gemv[k % blocks].replay()
+    e3.record(st)
+    e3.synchronize()
+    gemv_us = e2.elapsed_time(e3) * 1e3 / (reps * STEPS_PER_GRAPH)
+    gemv_us = max_over_ranks(gemv_us, world, device)
+
+    # end to end: pinned host activations in, output back to the host, every step
+    e_steps = max(STEPS_PER_GRAPH, min(args.steps, 16000) // STEPS_PER_GRAPH * STEPS_PER_GRAPH)
+    barrier(world, device)
+    torch.cuda.synchronize()
+    e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e4.record(st)
+    for k in range(e_steps // STEPS_PER_GRAPH):
+        g_e2e[k % blocks].replay()
+    e5.record(st)
+    e5.synchronize()
+    ms_e2e = max_over_ranks(e4.elapsed_time(e5), world, device) / e_steps
+
+    packed_bytes = layer.packed_bytes
+    value = world * packed_bytes / (ms_per_step * 1e-3) / 1e9
+    achieved = packed_bytes / (gemv_us * 1e-6) / 1e9
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    traffic = profiled_traffic("gemv_decode_lq24_10")
+    result = {
+        "metric": "decode GEMV packed-weight GB/s", "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "in": cfg.in_dim, "out": cfg.out, "d": cfg.d, "D": cfg.D,
+                   "K": cfg.K, "batch": 1, "tblk": cfg.tblk, "step": "lift + gemv",
+                   "l2": f"inputs larger than L2: {copies} rotating weight copies "
+                         f"({copies * per_copy / 1e6:.0f} MB vs L2 {l2 / 1e6:.0f} MB)",
+                   "parallelism": f"replicas{world}"},
+        "roofline": {"bound": "hbm", "kernel": "lq_gemv", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic, "peak_source": peaks_src,
+                     "avg_launch_us": gemv_us, "algorithmic_bytes_per_launch": packed_bytes},
+        "e2e": {"value": world * packed_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": int(layer.a[0].numel() * layer.a[0].element_size()),
+                "d2h_bytes_per_step": int(layer.o[0].numel() * 4), "ms_per_step": ms_e2e,
+                "note": "CUDA-graph replay of: H2D activations, lq_lift_activations, lq_gemv, D2H output"},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+
+    if rank == 0 and world == 1 and not args.no_extra:
+        extra = {}
+        extra["prefill_lq24_10"] = bench_prefill(torch, lq, "prefill_lq24_10", 2048)
+        extra["prefill_lq24_10"]["frac_of_bf16_peak"] = (
+            extra["prefill_lq24_10"]["gemm_TFLOPs"] / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])))
+        extra["decode_lq20_8"] = bench_decode_sweep(torch, lq, "decode_lq20_8", (1, 2, 4, 8, 16), l2)
+        for D in (16, 19, 20, 22, 24):
+            n = f"sweep_lq{D}_8"
+            extra[n] = {"b1": bench_decode_sweep(torch, lq, n, (1,), l2)["1"],
+                        "b64": bench_prefill(torch, lq, n, 64)}
+        result["extra"] = extra
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        nthreads = oracle.threads_available()
+        v, dt, desc = oracle_sample(args.workload, 15.0, nthreads)
+        result["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": nthreads, "kind": "oracle",
+                                  "sample": desc + f" ({dt:.1f} s)"}
+
+    assert lq.get_device_status() == lq.LQ_OK
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del g_full, g_single, g_gemv, g_e2e
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,160 @@
+"""Python binding of liblq.so, the C-ABI LiftQuant layer for B200 (sm_100a).
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels. PyTorch supplies device memory and the current stream. There is
+no fallback: if liblq.so is missing or cannot be loaded, import fails loudly.
+
+    o = diag(s) . W_q . (blockdiag(M^T) . T^{-1} . a)
+
+Entry points (same names as include/lq.h, minus the `lq_` prefix):
+    lifted_dim, pack_signs, unpack_signs, lift_activations, gemv, gemm,
+    get_device_status
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblq.so")
+
+LQ_OK, LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_TIMEOUT = 0, 1, 2, 3, 4
+LQ_F32, LQ_BF16 = 0, 1
+
+SYMBOLS = ("lq_status_str", "lq_lifted_dim", "lq_pack_signs", "lq_unpack_signs", "lq_lift_activations",
+           "lq_gemv", "lq_gemm", "lq_get_device_status")
+
+
+class LQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_str(status)}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"liblq.so not built at {LIB_PATH}; run `python -m bit_lifted_gemm_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    p, i = ctypes.c_void_p, ctypes.c_int
+    lib.lq_status_str.restype = ctypes.c_char_p
+    lib.lq_status_str.argtypes = [i]
+    lib.lq_lifted_dim.restype = i
+    lib.lq_lifted_dim.argtypes = [i, i, i]
+    lib.lq_pack_signs.restype = i
+    lib.lq_pack_signs.argtypes = [p, i, i, p, p]
+    lib.lq_unpack_signs.restype = i
+    lib.lq_unpack_signs.argtypes = [p, i, i, p, p]
+    lib.lq_lift_activations.restype = i
+    lib.lq_lift_activations.argtypes = [p, i, i, i, p, i, p, i, i, p, i, i, p]
+    lib.lq_gemv.restype = i
+    lib.lq_gemv.argtypes = [p, p, i, i, p, i, p, p]
+    lib.lq_gemm.restype = i
+    lib.lq_gemm.argtypes = [p, p, i, i, p, i, p, p]
+    lib.lq_get_device_status.restype = i
+    lib.lq_get_device_status.argtypes = [p]
+    return lib
+
+
+lib = _load()
+
+
+def status_str(status: int) -> str:
+    return lib.lq_status_str(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != LQ_OK:
+        raise LQError(status, where)
+
+
+def lifted_dim(in_dim: int, d: int, D: int) -> int:
+    return int(lib.lq_lifted_dim(in_dim, d, D))
+
+
+# ------------------------------------------------------------------ torch helpers
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev_tensor(t, name):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    return t
+
+
+def pack_signs(signs, out=None, stream=None):
+    """int8 +-1 [out][K] (CUDA) -> packed words [out][K/32] (int32 storage of uint32)."""
+    import torch
+    _dev_tensor(signs, "signs")
+    rows, K = signs.shape
+    if out is None:
+        out = torch.empty((rows, K // 32), dtype=torch.int32, device=signs.device)
+    _check(lib.lq_pack_signs(_ptr(signs), rows, K, _ptr(out), _stream(stream)), "lq_pack_signs")
+    return out
+
+
+def unpack_signs(packed, K, out=None, stream=None):
+    import torch
+    _dev_tensor(packed, "packed")
+    rows = packed.shape[0]
+    if out is None:
+        out = torch.empty((rows, K), dtype=torch.int8, device=packed.device)
+    _check(lib.lq_unpack_signs(_ptr(packed), rows, K, _ptr(out), _stream(stream)), "lq_unpack_signs")
+    return out
+
+
+def lift_activations(a, M, K, tinv=None, u_dtype="f32", out=None, stream=None):
+    """a [batch][in] (float32 or bfloat16) -> u [batch][K] (float32 or bfloat16)."""
+    import torch
+    _dev_tensor(a, "a")
+    _dev_tensor(M, "M")
+    batch, in_dim = a.shape
+    d, D = M.shape
+    a_t = LQ_BF16 if a.dtype == torch.bfloat16 else LQ_F32
+    u_t = LQ_BF16 if u_dtype in ("bf16", torch.bfloat16) else LQ_F32
+    if out is None:
+        out = torch.empty((batch, K), dtype=torch.bfloat16 if u_t == LQ_BF16 else torch.float32, device=a.device)
+    tblk = 0 if tinv is None else int(tinv.shape[-1])
+    if tinv is not None:
+        _dev_tensor(tinv, "tinv")
+    _check(lib.lq_lift_activations(_ptr(a), a_t, batch, in_dim, _ptr(tinv), tblk, _ptr(M), d, D, _ptr(out), u_t,
+                                   K, _stream(stream)), "lq_lift_activations")
+    return out
+
+
+def gemv(packed, s, u, out=None, stream=None):
+    """Decode: packed [out][K/32], s [out], u fp32 [batch][K] (batch <= 16) -> o fp32 [batch][out]."""
+    import torch
+    _dev_tensor(packed, "packed")
+    _dev_tensor(u, "u")
+    rows = packed.shape[0]
+    batch, K = u.shape
+    if out is None:
+        out = torch.empty((batch, rows), dtype=torch.float32, device=u.device)
+    _check(lib.lq_gemv(_ptr(packed), _ptr(s), rows, K, _ptr(u), batch, _ptr(out), _stream(stream)), "lq_gemv")
+    return out
+
+
+def gemm(packed, s, u, out=None, stream=None):
+    """Prefill: packed [out][K/32], s [out], u bf16 [tokens][K] -> o fp32 [tokens][out]."""
+    import torch
+    _dev_tensor(packed, "packed")
+    _dev_tensor(u, "u")
+    rows = packed.shape[0]
+    tokens, K = u.shape
+    if out is None:
+        out = torch.empty((tokens, rows), dtype=torch.float32, device=u.device)
+    _check(lib.lq_gemm(_ptr(packed), _ptr(s), rows, K, _ptr(u), tokens, _ptr(out), _stream(stream)), "lq_gemm")
+    return out
+
+
+def get_device_status(stream=None) -> int:
+    return int(lib.lq_get_device_status(_stream(stream)))

@@ -1,0 +1,138 @@
+// C ABI of the LiftQuant layer (declared in include/lq.h). This file validates
+// arguments synchronously, before any CUDA call, and enqueues the kernels on
+// the caller's stream. The only device state it owns is one status word per
+// device (a module-scope __device__ variable), which bounded waits in the
+// kernels set when they give up.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lq.h"
+#include "lq_internal.h"
+
+namespace {
+
+__device__ unsigned g_lq_status;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? LQ_OK : LQ_ERR_CUDA; }
+
+// Device address of the status word on the current device (looked up once per device).
+unsigned* status_word(int* err) {
+    static unsigned* addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) {
+        *err = LQ_ERR_CUDA;
+        return nullptr;
+    }
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_lq_status) != cudaSuccess) {
+            *err = LQ_ERR_CUDA;
+            return nullptr;
+        }
+        addr[dev] = static_cast<unsigned*>(p);
+    }
+    *err = LQ_OK;
+    return addr[dev];
+}
+
+// 1 if the current device is an sm_100 part, 0 if not, -1 on error (cached per device).
+int is_sm100() {
+    static signed char cache[kMaxDevices];
+    static bool init[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return -1;
+    if (!init[dev]) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return -1;
+        if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return -1;
+        cache[dev] = (major == 10 && minor == 0) ? 1 : 0;
+        init[dev] = true;
+    }
+    return cache[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lq_status_str(int status) {
+    switch (status) {
+        case LQ_OK: return "LQ_OK";
+        case LQ_ERR_INVALID_ARG: return "LQ_ERR_INVALID_ARG";
+        case LQ_ERR_UNSUPPORTED: return "LQ_ERR_UNSUPPORTED";
+        case LQ_ERR_CUDA: return "LQ_ERR_CUDA";
+        case LQ_ERR_TIMEOUT: return "LQ_ERR_TIMEOUT";
+        default: return "LQ_ERR_UNKNOWN";
+    }
+}
+
+int lq_lifted_dim(int in, int d, int D) {
+    if (in <= 0 || d <= 0 || D <= 0 || in % d != 0) return -1;
+    long long k = (long long)(in / d) * D;
+    k = (k + 31) / 32 * 32;
+    return k > 0x7fffffffLL ? -1 : (int)k;
+}
+
+int lq_pack_signs(const int8_t* signs_pm1, int out, int K, uint32_t* packed, void* stream) {
+    if (!signs_pm1 || !packed || !aligned16(signs_pm1) || !aligned16(packed)) return LQ_ERR_INVALID_ARG;
+    if (out < 1 || K < 32 || K % 32 != 0) return LQ_ERR_INVALID_ARG;
+    return from_cuda(lq::launch_pack(signs_pm1, out, K, packed, static_cast<cudaStream_t>(stream)));
+}
+
+int lq_unpack_signs(const uint32_t* packed, int out, int K, int8_t* signs_pm1, void* stream) {
+    if (!signs_pm1 || !packed || !aligned16(signs_pm1) || !aligned16(packed)) return LQ_ERR_INVALID_ARG;
+    if (out < 1 || K < 32 || K % 32 != 0) return LQ_ERR_INVALID_ARG;
+    return from_cuda(lq::launch_unpack(packed, out, K, signs_pm1, static_cast<cudaStream_t>(stream)));
+}
+
+int lq_lift_activations(const void* a, int a_dtype, int batch, int in, const float* tinv, int tblk,
+                        const float* M, int d, int D, void* u, int u_dtype, int K, void* stream) {
+    if (!a || !M || !u || !aligned16(a) || !aligned16(M) || !aligned16(u)) return LQ_ERR_INVALID_ARG;
+    if (tinv && !aligned16(tinv)) return LQ_ERR_INVALID_ARG;
+    if ((a_dtype != LQ_F32 && a_dtype != LQ_BF16) || (u_dtype != LQ_F32 && u_dtype != LQ_BF16))
+        return LQ_ERR_INVALID_ARG;
+    if (batch < 1 || in < 1 || d < 1 || d > 64 || D < 1 || D > 256 || d * D > 4096) return LQ_ERR_INVALID_ARG;
+    if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
+    if (tinv && (tblk < 1 || tblk > 256 || in % tblk != 0)) return LQ_ERR_INVALID_ARG;
+    return from_cuda(lq::launch_lift(a, a_dtype == LQ_BF16, batch, in, tinv, tblk, M, d, D, u, u_dtype == LQ_BF16,
+                                     K, static_cast<cudaStream_t>(stream)));
+}
+
+int lq_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u, int batch, float* o,
+            void* stream) {
+    if (!packed || !s || !u || !o) return LQ_ERR_INVALID_ARG;
+    if (!aligned16(packed) || !aligned16(s) || !aligned16(u) || !aligned16(o)) return LQ_ERR_INVALID_ARG;
+    if (out < 1 || K < 32 || K % 32 != 0 || batch < 1 || batch > 16) return LQ_ERR_INVALID_ARG;
+    return from_cuda(lq::launch_gemv(packed, s, out, K, u, batch, o, static_cast<cudaStream_t>(stream)));
+}
+
+int lq_gemm(const uint32_t* packed, const float* s, int out, int K, const uint16_t* u_bf16, int tokens, float* o,
+            void* stream) {
+    if (!packed || !s || !u_bf16 || !o) return LQ_ERR_INVALID_ARG;
+    if (!aligned16(packed) || !aligned16(s) || !aligned16(u_bf16) || !aligned16(o)) return LQ_ERR_INVALID_ARG;
+    if (out < 1 || K < 32 || K % 32 != 0 || tokens < 1) return LQ_ERR_INVALID_ARG;
+    const int sm = is_sm100();
+    if (sm < 0) return LQ_ERR_CUDA;
+    if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    int err = LQ_OK;
+    unsigned* status = status_word(&err);
+    if (!status) return err;
+    return from_cuda(lq::launch_gemm(packed, s, out, K, u_bf16, tokens, o, status, static_cast<cudaStream_t>(stream)));
+}
+
+int lq_get_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return LQ_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_lq_status, sizeof(v)) != cudaSuccess) return LQ_ERR_CUDA;
+    if (v) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_lq_status, &zero, sizeof(zero)) != cudaSuccess) return LQ_ERR_CUDA;
+    }
+    return (v & LQ_DEV_TIMEOUT) ? LQ_ERR_TIMEOUT : LQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,233 @@
+// Prefill 1-bit GEMM on the fifth-generation tensor cores (LiftQuant paper
+// note, "Key designs" 4: the layer is a 1-bit x float matmul with W_q after the
+// small matmul T* a, then diag(s)):
+//
+//   o[t][r] = s[r] * sum_k sigma[r][k] u[t][k]
+//
+// Prefill is a dense contraction, so it runs on tcgen05 with bf16 operands and
+// fp32 accumulation in tensor memory. +-1 is exact in bf16 and every product
+// is exact; the only rounding is fp32 accumulation (plus the bf16 rounding of
+// u done by the lift).
+//
+// One CTA computes a 128 (rows of W_q) x 256 (tokens) tile, K in steps of 64:
+//   warp 0      TMA producer: u tile [256 tokens][64 k] bf16, 128-byte swizzle
+//   warp 1      TMEM allocator and single-thread UMMA issuer (M=128, N=256, K=16)
+//   warps 2..5  one thread per tile row: load that row's two sign words for the
+//               k-step, expand the 64 bits to +-1 bf16 in registers and store
+//               them in the same 128-byte-swizzled K-major layout the TMA uses;
+//               after the K loop the same warps drain TMEM (tcgen05.ld), apply
+//               s[r] and store o.
+// A 4-stage mbarrier ring couples them; the unpackers fence the generic-proxy
+// stores into the async proxy before arriving. Every wait is bounded.
+#include <cuda.h>
+
+#include "lq_internal.h"
+#include "lq_sm100.cuh"
+
+namespace lq {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_STAGE = BM * BK * 2;   // 16 KB
+constexpr int B_STAGE = BN * BK * 2;   // 32 KB
+constexpr int TMEM_COLS = 256;         // fp32 accumulator, 128 lanes x 256 columns
+constexpr int THREADS = 192;
+constexpr int UNPACK_THREADS = 128;
+constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * (A_STAGE + B_STAGE) + 256;
+
+// Expand 16 sign bits (bit i = element i of a k-run) into 8 bf16x2 words:
+// word i holds elements (2i, 2i+1) as +1.0 (0x3F80) or -1.0 (0xBF80).
+// Even bits stay, odd bits move up by 15 so that one shift brings bits 2i and
+// 2i+1 to the two sign positions (15 and 31).
+__device__ __forceinline__ void expand16(uint32_t x, uint32_t* v) {
+    const uint32_t q = (x & 0x5555u) | ((x & 0xAAAAu) << 15);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = ((q << (15 - 2 * i)) & 0x80008000u) ^ 0xBF80BF80u;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_u, const uint32_t* __restrict__ packed,
+                const float* __restrict__ s, int out, int K, int tokens, float* __restrict__ o,
+                unsigned* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * A_STAGE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + STAGES), accf = smem_addr(bars + 2 * STAGES);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
+    const int nkb = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < STAGES; ++st) {
+            mbar_init(full0 + 8 * st, 1 + UNPACK_THREADS);
+            mbar_init(empty0 + 8 * st, 1);
+        }
+        mbar_init(accf, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tmap_u);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int st = kb % STAGES, round = kb / STAGES;
+                if (round > 0 && !mbar_wait(empty0 + 8 * st, (round - 1) & 1, status)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(full0 + 8 * st, B_STAGE);
+                tma_load_2d(smem_addr(sB + st * B_STAGE), &tmap_u, kb * BK, n0, full0 + 8 * st);
+                issued = kb + 1;
+            }
+            // Do not leave copies in flight: wait (bounded) for the last load of each stage.
+            for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
+                mbar_wait(full0 + 8 * (kb % STAGES), (kb / STAGES) & 1, status);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(BM, BN);
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int st = kb % STAGES, round = kb / STAGES;
+                if (!mbar_wait(full0 + 8 * st, round & 1, status)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_base = smem_addr(sA + st * A_STAGE), b_base = smem_addr(sB + st * B_STAGE);
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    umma_f16(tmem, smem_desc_sw128(a_base + kk * 32), smem_desc_sw128(b_base + kk * 32), idesc,
+                             (kb | kk) != 0);
+                umma_commit(empty0 + 8 * st);
+            }
+            umma_commit(accf);  // fires once every issued MMA has completed
+        }
+    } else {
+        // ---- unpack: thread `row` writes row `row` of every A stage
+        const int row = threadIdx.x - 64;
+        const int kw = K >> 5;
+        const int grow = m0 + row < out ? m0 + row : out - 1;  // rows past `out` are computed but never stored
+        const uint32_t* prow = packed + (long long)grow * kw;
+        const uint32_t sw = row & 7;
+        const uint32_t row_off = (row >> 3) * 1024 + (row & 7) * 128;
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int st = kb % STAGES, round = kb / STAGES;
+            const uint32_t w0 = 2 * kb < kw ? __ldg(prow + 2 * kb) : 0u;
+            const uint32_t w1 = 2 * kb + 1 < kw ? __ldg(prow + 2 * kb + 1) : 0u;  // u is zero past K
+            uint32_t v[32];
+            expand16(w0 & 0xFFFFu, v);
+            expand16(w0 >> 16, v + 8);
+            expand16(w1 & 0xFFFFu, v + 16);
+            expand16(w1 >> 16, v + 24);
+            if (round > 0 && !mbar_wait(empty0 + 8 * st, (round - 1) & 1, status)) {
+                *abort_flag = 1;
+                break;
+            }
+            const uint32_t dst = smem_addr(sA + st * A_STAGE) + row_off;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                st_shared_v4(dst + ((c ^ sw) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            fence_proxy_async_smem();
+            mbar_arrive(full0 + 8 * st);
+        }
+
+        // ---- epilogue: TMEM -> registers -> s[r] * acc -> o[t][r]
+        const bool done = mbar_wait(accf, 0, status);
+        tc_fence_after();
+        // tcgen05.ld is warp-collective: decide for the whole warp at once
+        if (__all_sync(0xffffffffu, done && !*abort_flag)) {
+            const int q = warp & 3;  // this warp's TMEM lane quadrant
+            const int m = m0 + q * 32 + lane;
+            const float sr = m < out ? __ldg(s + m) : 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + c0, v);
+                tmem_ld_wait();
+                if (m < out) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = n0 + c0 + j;
+                        if (n < tokens) o[(long long)n * out + m] = sr * __uint_as_float(v[j]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const uint32_t* packed, const float* s, int out, int K, const uint16_t* u_bf16,
+                        int tokens, float* o, unsigned* status, cudaStream_t st) {
+    EncodeTiledFn encode = encode_fn();
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap map;
+    cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)tokens};
+    cuuint64_t gstride[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {BK, BN};
+    cuuint32_t estride[2] = {1, 1};
+    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(u_bf16), gdim, gstride, box,
+                        estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    dim3 grid((out + BM - 1) / BM, (tokens + BN - 1) / BN);
+    gemm_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(map, packed, s, out, K, tokens, o, status);
+    return cudaGetLastError();
+}
+
+}  // namespace lq

@@ -1,0 +1,28 @@
+// Internal launchers of the LiftQuant sm_100a kernels. Each returns the
+// cudaError_t of its launch; argument validation happens in lq_api.cu before
+// any of these is called.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+// Bits of the device status word (read and cleared by lq_get_device_status).
+#define LQ_DEV_TIMEOUT 1u
+
+namespace lq {
+
+cudaError_t launch_pack(const int8_t* signs, int out, int K, uint32_t* packed, cudaStream_t st);
+cudaError_t launch_unpack(const uint32_t* packed, int out, int K, int8_t* signs, cudaStream_t st);
+
+cudaError_t launch_lift(const void* a, bool a_bf16, int batch, int in, const float* tinv, int tblk,
+                        const float* M, int d, int D, void* u, bool u_bf16, int K, cudaStream_t st);
+
+cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u,
+                        int batch, float* o, cudaStream_t st);
+
+// Prefill GEMM on tcgen05. `status` is the device status word.
+cudaError_t launch_gemm(const uint32_t* packed, const float* s, int out, int K,
+                        const uint16_t* u_bf16, int tokens, float* o, unsigned* status,
+                        cudaStream_t st);
+
+}  // namespace lq

@@ -14,6 +14,8 @@ from .inputs import (  # noqa: F401
     f32_from_bf16_bits,
     make_layer,
     make_signs_pm1,
+    make_packed_random,
     make_u_bf16,
+    make_u_f32,
     rng_for,
 )

@@ -108,6 +108,11 @@ def make_u_bf16(tokens: int, K: int, cfg_index: int, extra: int = 0) -> np.ndarr
     return bf16_bits_from_f32(g.standard_normal((tokens, K)).astype(np.float32))
 
 
+def make_u_f32(batch: int, K: int, cfg_index: int, extra: int = 0) -> np.ndarray:
+    """Lifted activations drawn directly, N(0, 1) in fp32."""
+    return rng_for(cfg_index, LIFTED, extra).standard_normal((batch, K)).astype(np.float32)
+
+
 def _orthogonal_blocks(nblk: int, tblk: int, g: np.random.Generator) -> np.ndarray:
     out = np.empty((nblk, tblk, tblk), dtype=np.float32)
     for b in range(nblk):

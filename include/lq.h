@@ -1,0 +1,116 @@
+/*
+ * lq.h -- C ABI of the LiftQuant lift-then-project layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer (LiftQuant: Continuous Bit-Width LLM via Dimensional Lifting and
+ * Projection, ICML 2026; paper note "Key designs" 1, 3 and 4) computes
+ *
+ *     o = diag(s) . W_q . (blockdiag(M^T) . T^{-1} . a)
+ *
+ * with W_q in {+-1}^{out x K} stored as packed sign bits, M in R^{d x D} the
+ * global projection, T^{-1} the per-layer whitening inverse and
+ * K = (in/d)*D rounded up to a multiple of 32, so the weight bit-width is D/d.
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are caller-owned DEVICE memory, 16-byte aligned,
+ *    densely packed row-major. The library frees nothing and keeps no pointer.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *    stream-ordered and asynchronous: they return after enqueueing work.
+ *  - Argument checks are synchronous and happen before any launch; a call
+ *    that fails them launches nothing and returns LQ_ERR_INVALID_ARG.
+ *  - A failed launch returns LQ_ERR_CUDA. Errors detected on the device
+ *    (a bounded wait that ran out) are latched in a device status word read
+ *    by lq_get_device_status().
+ *  - Packed signs: 32 per uint32, least significant bit first along the
+ *    lifted axis, bit 1 = +1, row-major [out][K/32].
+ *  - bf16 values are passed as their uint16 bit patterns.
+ */
+#ifndef LQ_H
+#define LQ_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LQ_API __attribute__((visibility("default")))
+#else
+#define LQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LQ_OK = 0,
+    LQ_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or dtype; nothing launched */
+    LQ_ERR_UNSUPPORTED = 2,  /* valid but not supported on this device (needs sm_100) */
+    LQ_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+    LQ_ERR_TIMEOUT = 4       /* a device-side bounded wait expired (from lq_get_device_status) */
+} lq_status;
+
+typedef enum { LQ_F32 = 0, LQ_BF16 = 1 } lq_dtype;
+
+/* Human-readable name of a status code; never NULL. */
+LQ_API const char* lq_status_str(int status);
+
+/* Lifted width K = (in/d)*D rounded up to a multiple of 32 (storage of D sign
+ * bits per d weights, "Key designs" 1). Returns -1 if d does not divide in or
+ * an argument is not positive or the result overflows int. Host only. */
+LQ_API int lq_lifted_dim(int in, int d, int D);
+
+/* Pack +-1 signs into words (the 1-bit W_q of "Key designs" 4).
+ *   signs_pm1 : int8 [out][K], each +1 or -1 (any value > 0 packs as 1)
+ *   out >= 1, K >= 32 and K % 32 == 0
+ *   packed    : uint32 [out][K/32] (written)
+ * Bit-exact. */
+LQ_API int lq_pack_signs(const int8_t* signs_pm1, int out, int K, uint32_t* packed, void* stream);
+
+/* Inverse of lq_pack_signs: words -> int8 +-1 [out][K]. Bit-exact. */
+LQ_API int lq_unpack_signs(const uint32_t* packed, int out, int K, int8_t* signs_pm1, void* stream);
+
+/* Activation lift u = blockdiag(M^T) . T^{-1} . a  (the small matmul T* a
+ * computed once before the 1-bit matmul, "Key designs" 4; T on the activation
+ * side, "Key designs" 3).
+ *   a      : [batch][in], a_dtype LQ_F32 or LQ_BF16
+ *   tinv   : fp32 [in/tblk][tblk][tblk], block-diagonal T^{-1}, block b maps
+ *            channels [b*tblk, (b+1)*tblk); NULL means T = identity (tblk ignored)
+ *            1 <= tblk <= 256, in % tblk == 0
+ *   M      : fp32 [d][D]; in % d == 0, 1 <= d <= 64, 1 <= D <= 256, d*D <= 4096
+ *   u      : [batch][K] written in u_dtype: LQ_F32 (decode) or LQ_BF16 (prefill,
+ *            round to nearest even); u[c][b*D + j] = sum_i M[i][j] a'[c][b*d + i]
+ *            with a' = T^{-1} a; entries at (in/d)*D .. K-1 are written as 0
+ *   K      : must equal lq_lifted_dim(in, d, D); batch >= 1
+ * Accumulation is fp32. */
+LQ_API int lq_lift_activations(const void* a, int a_dtype, int batch, int in,
+                        const float* tinv, int tblk,
+                        const float* M, int d, int D,
+                        void* u, int u_dtype, int K, void* stream);
+
+/* Decode 1-bit GEMV, batch 1..16 ("1-bit x float standard GEMM", "Key designs" 4):
+ *   o[c][r] = s[r] * sum_k sigma[r][k] * u[c][k],  sigma = +1 if bit set else -1
+ *   packed : uint32 [out][K/32]; s : fp32 [out]; u : fp32 [batch][K]
+ *   o      : fp32 [batch][out] (written)
+ *   out >= 1, K >= 32, K % 32 == 0, 1 <= batch <= 16
+ * Result within 1e-5 relative (Frobenius) of the exact value. */
+LQ_API int lq_gemv(const uint32_t* packed, const float* s, int out, int K,
+            const float* u, int batch, float* o, void* stream);
+
+/* Prefill 1-bit GEMM on the tensor cores (tcgen05, bf16 operands, fp32 accumulate):
+ *   o[t][r] = s[r] * sum_k sigma[r][k] * u[t][k]
+ *   packed : uint32 [out][K/32]; s : fp32 [out]; u_bf16 : bf16 bits [tokens][K]
+ *   o      : fp32 [tokens][out] (written)
+ *   out >= 1, K >= 32, K % 32 == 0, tokens >= 1
+ * +-1 is exact in bf16 and products are exact, so the only rounding is fp32
+ * accumulation. Requires an sm_100 device (else LQ_ERR_UNSUPPORTED). */
+LQ_API int lq_gemm(const uint32_t* packed, const float* s, int out, int K,
+            const uint16_t* u_bf16, int tokens, float* o, void* stream);
+
+/* Synchronizes `stream`, then returns and clears the device status word of the
+ * current device: LQ_OK, or LQ_ERR_TIMEOUT if a kernel gave up a bounded wait
+ * since the last call. Returns LQ_ERR_CUDA if the synchronize fails. */
+LQ_API int lq_get_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LQ_H */

@@ -1,0 +1,83 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/lq.h declares, and rejects bad arguments synchronously
+(before any CUDA call) with LQ_ERR_INVALID_ARG."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "lq.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"LQ_API\s+[\w\s\*]+?\b(lq_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    import bit_lifted_gemm_b200 as lq
+    declared = _declared_symbols()
+    assert len(declared) >= 8
+    assert set(declared) == set(lq.SYMBOLS)
+    for name in declared:
+        assert hasattr(lq.lib, name), name
+    with open(os.path.join(ROOT, "bit_lifted_gemm_b200", "liblq.so"), "rb") as f:
+        blob = f.read()
+    for name in declared:
+        assert name.encode() in blob
+
+
+def test_status_strings():
+    import bit_lifted_gemm_b200 as lq
+    assert lq.status_str(0) == "LQ_OK"
+    assert lq.status_str(1) == "LQ_ERR_INVALID_ARG"
+    assert lq.status_str(4) == "LQ_ERR_TIMEOUT"
+    assert lq.status_str(99) == "LQ_ERR_UNKNOWN"
+
+
+def test_lifted_dim_matches_oracle_closed_form():
+    import bit_lifted_gemm_b200 as lq
+    for args in [(640, 10, 24), (5120, 10, 24), (8192, 8, 20), (4096, 8, 19), (9, 3, 5), (10, 3, 5),
+                 (0, 1, 1), (7, 7, 1), (1 << 30, 1, 4)]:
+        assert lq.lifted_dim(*args) == oracle.lifted_dim(*args), args
+
+
+P = 0x100000  # a 16-byte-aligned fake address; never dereferenced (validation fails first)
+MIS = P + 4   # misaligned
+
+
+def _c(v):
+    return ctypes.c_void_p(v)
+
+
+@pytest.mark.parametrize("case", [
+    ("pack null", "lq_pack_signs", [None, 4, 32, _c(P), None]),
+    ("pack K%32", "lq_pack_signs", [_c(P), 4, 48, _c(P), None]),
+    ("pack out<1", "lq_pack_signs", [_c(P), 0, 32, _c(P), None]),
+    ("pack misaligned", "lq_pack_signs", [_c(MIS), 4, 32, _c(P), None]),
+    ("unpack null", "lq_unpack_signs", [_c(P), 4, 32, None, None]),
+    ("gemv batch 0", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 0, _c(P), None]),
+    ("gemv batch 17", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 17, _c(P), None]),
+    ("gemv K%32", "lq_gemv", [_c(P), _c(P), 8, 40, _c(P), 1, _c(P), None]),
+    ("gemv misaligned u", "lq_gemv", [_c(P), _c(P), 8, 64, _c(MIS), 1, _c(P), None]),
+    ("gemv null s", "lq_gemv", [_c(P), None, 8, 64, _c(P), 1, _c(P), None]),
+    ("gemm tokens 0", "lq_gemm", [_c(P), _c(P), 8, 64, _c(P), 0, _c(P), None]),
+    ("gemm K<32", "lq_gemm", [_c(P), _c(P), 8, 0, _c(P), 4, _c(P), None]),
+    ("gemm null o", "lq_gemm", [_c(P), _c(P), 8, 64, _c(P), 4, None, None]),
+    ("lift K mismatch", "lq_lift_activations", [_c(P), 0, 1, 640, None, 0, _c(P), 10, 24, _c(P), 0, 1504, None]),
+    ("lift d does not divide in", "lq_lift_activations", [_c(P), 0, 1, 641, None, 0, _c(P), 10, 24, _c(P), 0, 1536, None]),
+    ("lift tblk does not divide in", "lq_lift_activations", [_c(P), 1, 1, 640, _c(P), 96, _c(P), 10, 24, _c(P), 0, 1536, None]),
+    ("lift tblk too big", "lq_lift_activations", [_c(P), 1, 1, 1024, _c(P), 512, _c(P), 8, 16, _c(P), 0, 2048, None]),
+    ("lift bad dtype", "lq_lift_activations", [_c(P), 7, 1, 640, None, 0, _c(P), 10, 24, _c(P), 0, 1536, None]),
+    ("lift d too big", "lq_lift_activations", [_c(P), 0, 1, 130, None, 0, _c(P), 65, 2, _c(P), 0, 32, None]),
+    ("lift batch 0", "lq_lift_activations", [_c(P), 0, 0, 640, None, 0, _c(P), 10, 24, _c(P), 0, 1536, None]),
+], ids=lambda c: c[0])
+def test_invalid_arguments_rejected_before_launch(case):
+    import bit_lifted_gemm_b200 as lq
+    _, fn, args = case
+    assert getattr(lq.lib, fn)(*args) == lq.LQ_ERR_INVALID_ARG

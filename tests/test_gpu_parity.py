@@ -1,0 +1,248 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Tolerances: sign packing is bit-exact; the fp32 lift within 1e-6 relative; the
+decode GEMV within 1e-5 relative (Frobenius over [batch][out]); the prefill
+GEMM within 1e-5 of the oracle fed the same bf16 u (fp32 accumulation only)
+and within 5e-3 of the full-precision layer (bf16 rounding of u). Integer
+valued inputs make every sum exact, so the GPU must then match bit for bit.
+Full-size layers are checked on sampled rows that the oracle computes one by
+one, plus properties that hold at any size.
+"""
+
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from datagen import CONFIGS, make_layer, make_packed_random, make_signs_pm1, make_u_bf16, make_u_f32, rng_for
+from tests.gpu_common import dev, host, rel_err
+
+pytestmark = pytest.mark.gpu
+
+NTHREADS = min(32, oracle.threads_available())
+
+
+@pytest.fixture(scope="module")
+def lq():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import bit_lifted_gemm_b200 as lq
+    yield lq
+    assert lq.get_device_status() == lq.LQ_OK
+
+
+def _sample_rows(out, n, seed):
+    g = rng_for(77, 9, seed)
+    rows = np.unique(np.concatenate([g.choice(out, size=min(n, out), replace=False), [0, out - 1]]))
+    return rows.astype(np.int64)
+
+
+# ------------------------------------------------------------------ pack / unpack
+
+@pytest.mark.parametrize("rows,K", [(1, 32), (37, 288), (512, 1536), (1000, 12288)])
+def test_pack_unpack_bit_exact(lq, rows, K):
+    signs = make_signs_pm1(rows, K, cfg_index=50, extra=K)
+    packed = lq.pack_signs(dev(signs))
+    assert np.array_equal(host(packed), oracle.pack_signs(signs))
+    back = lq.unpack_signs(packed, K)
+    assert np.array_equal(host(back), signs)
+
+
+def test_pack_adversarial_patterns(lq):
+    K = 96
+    pats = np.stack([-np.ones(K), np.ones(K), np.tile([1, -1], K // 2), np.tile([-1, 1], K // 2),
+                     np.where(np.arange(K) % 32 == 31, 1, -1), np.where(np.arange(K) % 32 == 0, 1, -1)])
+    signs = pats.astype(np.int8)
+    assert np.array_equal(host(lq.pack_signs(dev(signs))), oracle.pack_signs(signs))
+    words = make_packed_random(8, 1024, cfg_index=51)
+    assert np.array_equal(host(lq.unpack_signs(dev(words), 1024)), oracle.unpack_signs(words, 1024))
+
+
+# ------------------------------------------------------------------ lift
+
+def _oracle_u(L):
+    a = oracle.to_f64(L.a, L.a_dtype)
+    t = None if L.tinv is None else oracle.to_f64(L.tinv)
+    return oracle.lift(oracle.whiten(a, t), oracle.to_f64(L.M), L.cfg.K)
+
+
+def _gpu_u(lq, L, u_dtype="f32"):
+    t = None if L.tinv is None else dev(L.tinv)
+    return lq.lift_activations(dev(L.a), dev(L.M), L.cfg.K, tinv=t, u_dtype=u_dtype)
+
+
+@pytest.mark.parametrize("name,batch", [("tiny", 1), ("tiny", 4), ("decode_lq24_10", 1), ("decode_lq20_8", 16),
+                                        ("decode_lq20_8", 3), ("sweep_lq19_8", 1)])
+def test_lift_fp32(lq, name, batch):
+    L = make_layer(CONFIGS[name], batch, packed=False)
+    u = host(_gpu_u(lq, L))
+    want = _oracle_u(L)
+    assert rel_err(u, want) <= 1e-6
+    assert np.max(np.abs(u - want)) <= 1e-5 * np.max(np.abs(want))
+
+
+def _bf16_ulp(x):
+    e = np.floor(np.log2(np.maximum(np.abs(x), 1e-30)))
+    return 2.0 ** (e - 7)
+
+
+@pytest.mark.parametrize("batch", [40, 100])
+def test_lift_bf16_prefill_tiles(lq, batch):
+    """Prefill variant (32-token tiles, ragged last tile), bf16 output."""
+    L = make_layer(CONFIGS["decode_lq24_10"], batch, packed=False)
+    u = oracle.to_f64(host(_gpu_u(lq, L, "bf16")), "bf16")
+    want = _oracle_u(L)
+    assert np.all(np.abs(u - want) <= _bf16_ulp(want) + 1e-6 * np.max(np.abs(want)))
+    assert rel_err(u, want) <= 3e-3
+
+
+def test_lift_padding_and_small_blocks(lq):
+    """in=9, d=3, D=5: K = 32 with 17 padded zeros; 3x3 whitening blocks."""
+    g = rng_for(60, 0)
+    a = g.standard_normal((2, 9)).astype(np.float32)
+    M = g.standard_normal((3, 5)).astype(np.float32)
+    tinv = g.standard_normal((3, 3, 3)).astype(np.float32)
+    for t in (None, tinv):
+        u = host(lq.lift_activations(dev(a), dev(M), 32, tinv=None if t is None else dev(t)))
+        want = oracle.lift(oracle.whiten(oracle.to_f64(a), None if t is None else oracle.to_f64(t)),
+                           oracle.to_f64(M), 32)
+        assert np.all(u[:, 15:] == 0.0)
+        assert rel_err(u, want) <= 1e-6
+
+
+# ------------------------------------------------------------------ decode GEMV
+
+@pytest.mark.parametrize("batch", [1, 4])
+def test_tiny_layer_full_path(lq, batch):
+    L = make_layer(CONFIGS["tiny"], batch)
+    u = _gpu_u(lq, L)
+    o = host(lq.gemv(dev(L.packed), dev(L.s), u))
+    _, want = oracle.forward(L.packed, L.s, oracle.to_f64(L.a), None, oracle.to_f64(L.M), L.cfg.K)
+    assert rel_err(o, want) <= 1e-5
+
+
+@pytest.mark.parametrize("out,K,batch", [(1000, 1536, 1), (1000, 1536, 3), (33, 1632, 16), (1, 32, 1),
+                                         (4097, 20480, 2), (700, 16384 + 1024, 1)])
+def test_gemv_ragged_vs_oracle(lq, out, K, batch):
+    packed = make_packed_random(out, K, 52, extra=K + out)
+    s = rng_for(52, 1, out).uniform(0.01, 0.03, out).astype(np.float32)
+    u = make_u_f32(batch, K, 52, extra=K)
+    o = host(lq.gemv(dev(packed), dev(s), dev(u)))
+    want = oracle.contract(packed, s, oracle.to_f64(u), NTHREADS)
+    assert rel_err(o, want) <= 1e-5
+
+
+def test_gemv_integer_inputs_exact(lq):
+    g = rng_for(53, 5)
+    out, K, batch = 777, 3072, 5
+    packed = make_packed_random(out, K, 53)
+    s = np.ones(out, dtype=np.float32)
+    u = g.integers(-8, 9, size=(batch, K)).astype(np.float32)
+    o = host(lq.gemv(dev(packed), dev(s), dev(u)))
+    want = oracle.contract(packed, s, oracle.to_f64(u))
+    assert np.array_equal(o.astype(np.float64), want)
+
+
+@pytest.mark.parametrize("D", [12, 16])
+def test_gemv_exhaustive_codebook(lq, D):
+    """One block, one row per sign pattern y in {+-1}^D: every codeword's output."""
+    d = 8
+    rows = 1 << D
+    packed = np.arange(rows, dtype=np.uint32).reshape(rows, 1)   # row r = pattern r, K = 32
+    g = rng_for(54, 2, D)
+    M = (g.standard_normal((d, D)) / np.sqrt(D)).astype(np.float32)
+    a = g.standard_normal((1, d)).astype(np.float32)
+    s = np.ones(rows, dtype=np.float32)
+    u = lq.lift_activations(dev(a), dev(M), 32)
+    o = host(lq.gemv(dev(packed), dev(s), u))
+    _, want = oracle.forward(packed, s, oracle.to_f64(a), None, oracle.to_f64(M), 32)
+    assert rel_err(o, want) <= 1e-5
+    # codeword identity: o[r] = (M y_r) . a for every pattern (dense reconstruction route)
+    want2 = oracle.dense_route(packed, s, oracle.to_f64(M), oracle.to_f64(a), 32)
+    assert rel_err(o, want2) <= 1e-5
+
+
+def test_decode_lq24_10_full_size(lq):
+    L = make_layer(CONFIGS["decode_lq24_10"], 1)
+    u = _gpu_u(lq, L)
+    o = host(lq.gemv(dev(L.packed), dev(L.s), u))
+    _, want = oracle.forward(L.packed, L.s, oracle.to_f64(L.a, "bf16"), oracle.to_f64(L.tinv),
+                             oracle.to_f64(L.M), L.cfg.K, NTHREADS)
+    assert rel_err(o, want) <= 1e-5
+
+
+@pytest.mark.parametrize("batch", [1, 2, 4, 8, 16])
+def test_decode_lq20_8_sampled_rows(lq, batch):
+    L = make_layer(CONFIGS["decode_lq20_8"], batch)
+    u = _gpu_u(lq, L)
+    o = host(lq.gemv(dev(L.packed), dev(L.s), u))
+    uref = _oracle_u(L)
+    rows = _sample_rows(L.cfg.out, 384, batch)
+    want = oracle.contract_rows(L.packed, L.s, uref, rows)
+    assert rel_err(o[:, rows], want) <= 1e-5
+    # whole-output property: E[o_r^2] = s_r^2 |u|^2 for iid signs
+    ratio = np.mean((o / L.s[None, :]) ** 2, axis=1) / np.sum(uref ** 2, axis=1)
+    assert np.all(np.abs(ratio - 1) < 0.05)
+
+
+@pytest.mark.parametrize("D", [16, 19, 20, 22, 24])
+def test_sweep_decode_sampled_rows(lq, D):
+    L = make_layer(CONFIGS[f"sweep_lq{D}_8"], 1)
+    u = _gpu_u(lq, L)
+    o = host(lq.gemv(dev(L.packed), dev(L.s), u))
+    rows = _sample_rows(L.cfg.out, 512, D)
+    want = oracle.contract_rows(L.packed, L.s, _oracle_u(L), rows)
+    assert rel_err(o[:, rows], want) <= 1e-5
+
+
+# ------------------------------------------------------------------ prefill GEMM
+
+@pytest.mark.parametrize("out,K,tokens", [(300, 1536, 300), (128, 64, 256), (129, 1568, 7), (1, 32, 1),
+                                          (517, 4096 + 32, 513)])
+def test_gemm_isolated_vs_oracle(lq, out, K, tokens):
+    packed = make_packed_random(out, K, 55, extra=K + out)
+    s = rng_for(55, 1, out).uniform(0.01, 0.03, out).astype(np.float32)
+    u = make_u_bf16(tokens, K, 55, extra=K + tokens)
+    o = host(lq.gemm(dev(packed), dev(s), dev(u)))
+    want = oracle.contract(packed, s, oracle.to_f64(u, "bf16"), NTHREADS)
+    assert rel_err(o, want) <= 1e-5
+
+
+def test_gemm_integer_inputs_exact(lq):
+    g = rng_for(56, 5)
+    out, K, tokens = 260, 2048, 300
+    packed = make_packed_random(out, K, 56)
+    s = np.ones(out, dtype=np.float32)
+    from datagen import bf16_bits_from_f32
+    u = bf16_bits_from_f32(g.integers(-8, 9, size=(tokens, K)).astype(np.float32))
+    o = host(lq.gemm(dev(packed), dev(s), dev(u)))
+    want = oracle.contract(packed, s, oracle.to_f64(u, "bf16"), NTHREADS)
+    assert np.array_equal(o.astype(np.float64), want)
+
+
+def test_prefill_lq24_10_full_size_sampled(lq):
+    L = make_layer(CONFIGS["prefill_lq24_10"], 2048)
+    u = _gpu_u(lq, L, "bf16")
+    o = host(lq.gemm(dev(L.packed), dev(L.s), u))
+    rows = _sample_rows(L.cfg.out, 96, 3)
+    toks = np.sort(rng_for(77, 8).choice(2048, size=192, replace=False))
+    # contraction alone: oracle fed the same bf16 u
+    u_host = oracle.to_f64(host(u), "bf16")
+    want_c = oracle.contract_rows(L.packed, L.s, u_host[toks], rows)
+    assert rel_err(o[np.ix_(toks, rows)], want_c) <= 1e-5
+    # whole layer against full-precision u
+    a = oracle.to_f64(L.a, "bf16")[toks]
+    uref = oracle.lift(oracle.whiten(a, oracle.to_f64(L.tinv)), oracle.to_f64(L.M), L.cfg.K)
+    want = oracle.contract_rows(L.packed, L.s, uref, rows)
+    assert rel_err(o[np.ix_(toks, rows)], want) <= 5e-3
+
+
+@pytest.mark.parametrize("D", [16, 24])
+def test_sweep_prefill_b64(lq, D):
+    L = make_layer(CONFIGS[f"sweep_lq{D}_8"], 64)
+    u = _gpu_u(lq, L, "bf16")
+    o = host(lq.gemm(dev(L.packed), dev(L.s), u))
+    rows = _sample_rows(L.cfg.out, 256, D)
+    want = oracle.contract_rows(L.packed, L.s, _oracle_u(L), rows)
+    assert rel_err(o[:, rows], want) <= 5e-3
