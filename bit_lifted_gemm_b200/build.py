@@ -1,6 +1,8 @@
 """Build liblq.so (the C-ABI library of sm_100a kernels) in-tree with nvcc.
 
-    python -m bit_lifted_gemm_b200.build [--force] [--verbose-ptxas]
+    python bit_lifted_gemm_b200/build.py [--force] [--verbose-ptxas]
+
+(Run it by path: importing the package loads liblq.so.)
 """
 
 from __future__ import annotations

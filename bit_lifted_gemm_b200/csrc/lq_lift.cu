@@ -122,6 +122,21 @@ __global__ void __launch_bounds__(256) lift_decode_kernel(LiftArgs p) {
     float* as = Ms + ((p.d * p.D + 3) & ~3); // [span][DEC_TB]
     float* aps = as + span * DEC_TB;        // [C][DEC_TB]
 
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    // The T^{-1} rows dominate this kernel's HBM traffic: request each warp's
+    // first two rows (up to 256 floats each) before anything else.
+    const bool vec = p.tinv && (p.tblk & 3) == 0 && p.tblk <= 256;
+    float4 tpre[2][2];
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl)
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int ch = warp + sl * nwarps, j4 = lane + 32 * q;
+            tpre[sl][q] = (vec && ch < r.C && j4 < (p.tblk >> 2))
+                              ? __ldg(reinterpret_cast<const float4*>(p.tinv + (long long)(r.c0 + ch) * p.tblk) + j4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+
     for (int i = threadIdx.x; i < p.d * p.D; i += blockDim.x) Ms[i] = __ldg(p.M + i);
     for (int i = threadIdx.x; i < span * nt; i += blockDim.x) {
         int t = i / span, j = i - t * span;
@@ -129,9 +144,50 @@ __global__ void __launch_bounds__(256) lift_decode_kernel(LiftArgs p) {
     }
     __syncthreads();
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    if (vec) {
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl) {
+            const int ch = warp + sl * nwarps;
+            if (ch >= r.C) continue;  // warp-uniform
+            const int c = r.c0 + ch;
+            const int base = (c / p.tblk) * p.tblk - r.lo;
+            float acc[DEC_TB];
+#pragma unroll
+            for (int t = 0; t < DEC_TB; ++t) acc[t] = 0.f;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int j4 = lane + 32 * q;
+                if (j4 < (p.tblk >> 2)) {
+                    const float4 tv = tpre[sl][q];
+                    const float* a0 = as + (base + 4 * j4) * DEC_TB;
+#pragma unroll
+                    for (int t = 0; t < DEC_TB; ++t) {
+                        if (t < nt) {
+                            float s = acc[t];
+                            s = fmaf(tv.x, a0[t], s);
+                            s = fmaf(tv.y, a0[DEC_TB + t], s);
+                            s = fmaf(tv.z, a0[2 * DEC_TB + t], s);
+                            s = fmaf(tv.w, a0[3 * DEC_TB + t], s);
+                            acc[t] = s;
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < DEC_TB; ++t) {
+                if (t < nt) {
+                    float v = acc[t];
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                    if (lane == 0) aps[ch * DEC_TB + t] = v;
+                }
+            }
+        }
+    }
     if (p.tinv) {
-        for (int ch = warp; ch < r.C; ch += nwarps) {
+        // channels beyond the two preloaded per warp, or whitening blocks that are
+        // not float4-friendly
+        for (int ch = vec ? warp + 2 * nwarps : warp; ch < r.C; ch += nwarps) {
             const int c = r.c0 + ch;
             const int base = (c / p.tblk) * p.tblk - r.lo;
             const float* row = p.tinv + (long long)c * p.tblk;  // row (c mod tblk) of block c/tblk
