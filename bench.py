@@ -190,7 +190,6 @@ class DecodeLayer:
         self.u = [torch.empty((batch, cfg.K), dtype=torch.float32, device=dev) for _ in range(copies)]
         self.o = [torch.empty((batch, cfg.out), dtype=torch.float32, device=dev) for _ in range(copies)]
         self.o_host = [torch.empty((batch, cfg.out), dtype=torch.float32).pin_memory() for _ in range(copies)]
-        self.ws = torch.empty(max(16, lq.gemv_workspace_size(cfg.out, cfg.K, batch)), dtype=torch.uint8, device=dev)
         self.copies = copies
         self.lq = lq
 
@@ -199,12 +198,12 @@ class DecodeLayer:
         if with_copies:
             self.a[i].copy_(self.a_host[i], non_blocking=True)
         lq.lift_activations(self.a[i], self.M, c.K, tinv=self.tinv[i], out=self.u[i])
-        lq.gemv(self.packed[i], self.s[i], self.u[i], out=self.o[i], workspace=self.ws)
+        lq.gemv(self.packed[i], self.s[i], self.u[i], out=self.o[i])
         if with_copies:
             self.o_host[i].copy_(self.o[i], non_blocking=True)
 
     def gemv_only(self, i):
-        self.lq.gemv(self.packed[i], self.s[i], self.u[i], out=self.o[i], workspace=self.ws)
+        self.lq.gemv(self.packed[i], self.s[i], self.u[i], out=self.o[i])
 
     @property
     def packed_bytes(self):

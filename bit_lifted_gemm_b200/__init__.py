@@ -7,8 +7,8 @@ no fallback: if liblq.so is missing or cannot be loaded, import fails loudly.
     o = diag(s) . W_q . (blockdiag(M^T) . T^{-1} . a)
 
 Entry points (same names as include/lq.h, minus the `lq_` prefix):
-    lifted_dim, pack_signs, unpack_signs, lift_activations, gemv_workspace_size,
-    gemv, gemm, get_device_status
+    lifted_dim, pack_signs, unpack_signs, lift_activations, gemv, gemm,
+    get_device_status
 """
 
 from __future__ import annotations
@@ -23,7 +23,7 @@ LQ_OK, LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_TIMEOUT = 0, 
 LQ_F32, LQ_BF16 = 0, 1
 
 SYMBOLS = ("lq_status_str", "lq_lifted_dim", "lq_pack_signs", "lq_unpack_signs", "lq_lift_activations",
-           "lq_gemv_workspace_size", "lq_gemv", "lq_gemm", "lq_get_device_status")
+           "lq_gemv", "lq_gemm", "lq_get_device_status")
 
 
 class LQError(RuntimeError):
@@ -47,10 +47,8 @@ def _load() -> ctypes.CDLL:
     lib.lq_unpack_signs.argtypes = [p, i, i, p, p]
     lib.lq_lift_activations.restype = i
     lib.lq_lift_activations.argtypes = [p, i, i, i, p, i, p, i, i, p, i, i, p]
-    lib.lq_gemv_workspace_size.restype = ctypes.c_size_t
-    lib.lq_gemv_workspace_size.argtypes = [i, i, i]
     lib.lq_gemv.restype = i
-    lib.lq_gemv.argtypes = [p, p, i, i, p, i, p, p, ctypes.c_size_t, p]
+    lib.lq_gemv.argtypes = [p, p, i, i, p, i, p, p]
     lib.lq_gemm.restype = i
     lib.lq_gemm.argtypes = [p, p, i, i, p, i, p, p]
     lib.lq_get_device_status.restype = i
@@ -132,28 +130,16 @@ def lift_activations(a, M, K, tinv=None, u_dtype="f32", out=None, stream=None):
     return out
 
 
-def gemv_workspace_size(out_rows: int, K: int, batch: int) -> int:
-    return int(lib.lq_gemv_workspace_size(out_rows, K, batch))
-
-
-def gemv(packed, s, u, out=None, workspace=None, stream=None):
-    """Decode: packed [out][K/32], s [out], u fp32 [batch][K] (batch <= 16) -> o fp32 [batch][out].
-
-    `workspace` is a uint8 CUDA tensor of at least gemv_workspace_size bytes; one is
-    allocated per call when omitted (pass one in to keep allocations off the hot path).
-    """
+def gemv(packed, s, u, out=None, stream=None):
+    """Decode: packed [out][K/32], s [out], u fp32 [batch][K] (batch <= 16) -> o fp32 [batch][out]."""
     import torch
     _dev_tensor(packed, "packed")
     _dev_tensor(u, "u")
     rows = packed.shape[0]
     batch, K = u.shape
-    need = gemv_workspace_size(rows, K, batch)
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=u.device)
     if out is None:
         out = torch.empty((batch, rows), dtype=torch.float32, device=u.device)
-    _check(lib.lq_gemv(_ptr(packed), _ptr(s), rows, K, _ptr(u), batch, _ptr(out), _ptr(workspace),
-                       workspace.numel() * workspace.element_size(), _stream(stream)), "lq_gemv")
+    _check(lib.lq_gemv(_ptr(packed), _ptr(s), rows, K, _ptr(u), batch, _ptr(out), _stream(stream)), "lq_gemv")
     return out
 
 

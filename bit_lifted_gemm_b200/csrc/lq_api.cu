@@ -102,26 +102,18 @@ int lq_lift_activations(const void* a, int a_dtype, int batch, int in, const flo
                                      K, static_cast<cudaStream_t>(stream)));
 }
 
-size_t lq_gemv_workspace_size(int out, int K, int batch) {
-    if (out < 1 || K < 32 || K % 32 != 0 || batch < 1 || batch > 16) return 0;
-    return lq::gemv_workspace_size(out, K, batch);
-}
-
 int lq_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u, int batch, float* o,
-            void* workspace, size_t workspace_bytes, void* stream) {
-    if (!packed || !s || !u || !o || !workspace) return LQ_ERR_INVALID_ARG;
-    if (!aligned16(packed) || !aligned16(s) || !aligned16(u) || !aligned16(o) || !aligned16(workspace))
-        return LQ_ERR_INVALID_ARG;
+            void* stream) {
+    if (!packed || !s || !u || !o) return LQ_ERR_INVALID_ARG;
+    if (!aligned16(packed) || !aligned16(s) || !aligned16(u) || !aligned16(o)) return LQ_ERR_INVALID_ARG;
     if (out < 1 || K < 32 || K % 32 != 0 || batch < 1 || batch > 16) return LQ_ERR_INVALID_ARG;
-    if (workspace_bytes < lq::gemv_workspace_size(out, K, batch)) return LQ_ERR_INVALID_ARG;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
     int err = LQ_OK;
     unsigned* status = status_word(&err);
     if (!status) return err;
-    return from_cuda(
-        lq::launch_gemv(packed, s, out, K, u, batch, o, workspace, status, static_cast<cudaStream_t>(stream)));
+    return from_cuda(lq::launch_gemv(packed, s, out, K, u, batch, o, status, static_cast<cudaStream_t>(stream)));
 }
 
 int lq_gemm(const uint32_t* packed, const float* s, int out, int K, const uint16_t* u_bf16, int tokens, float* o,

@@ -18,11 +18,10 @@ cudaError_t launch_unpack(const uint32_t* packed, int out, int K, int8_t* signs,
 cudaError_t launch_lift(const void* a, bool a_bf16, int batch, int in, const float* tinv, int tblk,
                         const float* M, int d, int D, void* u, bool u_bf16, int K, cudaStream_t st);
 
-// Decode GEMV: quantizes u into `workspace` (gemv_workspace_size bytes), then
-// runs the integer tensor-core GEMV. `status` is the device status word.
-size_t gemv_workspace_size(int out, int K, int batch);
+// Decode GEMV (integer tensor cores; u quantized per CTA). `status` is the
+// device status word that bounded waits report to.
 cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u,
-                        int batch, float* o, void* workspace, unsigned* status, cudaStream_t st);
+                        int batch, float* o, unsigned* status, cudaStream_t st);
 
 // Prefill GEMM on tcgen05. `status` is the device status word.
 cudaError_t launch_gemm(const uint32_t* packed, const float* s, int out, int K,

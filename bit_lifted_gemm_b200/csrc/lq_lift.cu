@@ -113,6 +113,9 @@ __device__ __forceinline__ void lift_and_store(const LiftArgs& p, const Range& r
 constexpr int DEC_TB = 16;
 
 __global__ void __launch_bounds__(256) lift_decode_kernel(LiftArgs p) {
+    // A programmatically dependent consumer (the decode GEMV) may start now: it
+    // streams its weights and waits for this grid before reading u.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ float smem[];
     const Range r = cta_range(p);
     const int t0 = blockIdx.y * DEC_TB;
@@ -243,6 +246,7 @@ constexpr int PRE_TB = 32;  // tokens per CTA
 constexpr int PRE_TT = 8;   // tokens per thread
 
 __global__ void __launch_bounds__(256) lift_prefill_kernel(LiftArgs p) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // see lift_decode_kernel
     extern __shared__ float smem[];
     const Range r = cta_range(p);
     const int t0 = blockIdx.y * PRE_TB;

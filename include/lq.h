@@ -27,7 +27,6 @@
 #ifndef LQ_H
 #define LQ_H
 
-#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -86,26 +85,18 @@ LQ_API int lq_lift_activations(const void* a, int a_dtype, int batch, int in,
                         const float* M, int d, int D,
                         void* u, int u_dtype, int K, void* stream);
 
-/* Bytes of device workspace lq_gemv needs for this shape; 0 if the arguments
- * are invalid (same checks as lq_gemv). Host only. */
-LQ_API size_t lq_gemv_workspace_size(int out, int K, int batch);
-
 /* Decode 1-bit GEMV, batch 1..16 ("1-bit x float standard GEMM", "Key designs" 4):
  *   o[c][r] = s[r] * sum_k sigma[r][k] * u[c][k],  sigma = +1 if bit set else -1
  *   packed : uint32 [out][K/32]; s : fp32 [out]; u : fp32 [batch][K]
  *   o      : fp32 [batch][out] (written)
- *   workspace : caller-owned device scratch of at least
- *               lq_gemv_workspace_size(out, K, batch) bytes, 16-byte aligned; it
- *               needs no initialization and holds nothing between calls, but
- *               two calls that may run concurrently must not share it
  *   out >= 1, K >= 32, K % 32 == 0, 1 <= batch <= 16
  * u is converted per K-part and column to 24-bit fixed point (error <= 2^-22 of
  * the part's largest |u|); the sign contraction itself is exact integer
  * arithmetic, so the result is within ~1e-6 relative (Frobenius) of the exact
- * value. Deterministic. Requires an sm_100 device (else LQ_ERR_UNSUPPORTED). */
+ * value. Deterministic. Needs no scratch memory. Requires an sm_100 device
+ * (else LQ_ERR_UNSUPPORTED). */
 LQ_API int lq_gemv(const uint32_t* packed, const float* s, int out, int K,
-            const float* u, int batch, float* o,
-            void* workspace, size_t workspace_bytes, void* stream);
+            const float* u, int batch, float* o, void* stream);
 
 /* Prefill 1-bit GEMM on the tensor cores (tcgen05, bf16 operands, fp32 accumulate):
  *   o[t][r] = s[r] * sum_k sigma[r][k] * u[t][k]

@@ -32,16 +32,6 @@ def test_library_exports_every_declared_symbol():
         assert name.encode() in blob
 
 
-def test_gemv_workspace_size():
-    import bit_lifted_gemm_b200 as lq
-    assert lq.gemv_workspace_size(13824, 12288, 1) >= 3 * 12288  # three digit planes per lifted element
-    assert lq.gemv_workspace_size(28672, 20480, 16) >= 3 * 16 * 20480
-    assert lq.gemv_workspace_size(8, 40, 1) == 0
-    assert lq.gemv_workspace_size(8, 64, 0) == 0
-    assert lq.gemv_workspace_size(8, 64, 17) == 0
-    assert lq.gemv_workspace_size(0, 64, 1) == 0
-
-
 def test_status_strings():
     import bit_lifted_gemm_b200 as lq
     assert lq.status_str(0) == "LQ_OK"
@@ -71,14 +61,11 @@ def _c(v):
     ("pack out<1", "lq_pack_signs", [_c(P), 0, 32, _c(P), None]),
     ("pack misaligned", "lq_pack_signs", [_c(MIS), 4, 32, _c(P), None]),
     ("unpack null", "lq_unpack_signs", [_c(P), 4, 32, None, None]),
-    ("gemv batch 0", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 0, _c(P), _c(P), 1 << 20, None]),
-    ("gemv batch 17", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 17, _c(P), _c(P), 1 << 20, None]),
-    ("gemv K%32", "lq_gemv", [_c(P), _c(P), 8, 40, _c(P), 1, _c(P), _c(P), 1 << 20, None]),
-    ("gemv misaligned u", "lq_gemv", [_c(P), _c(P), 8, 64, _c(MIS), 1, _c(P), _c(P), 1 << 20, None]),
-    ("gemv null s", "lq_gemv", [_c(P), None, 8, 64, _c(P), 1, _c(P), _c(P), 1 << 20, None]),
-    ("gemv null workspace", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 1, _c(P), None, 1 << 20, None]),
-    ("gemv workspace too small", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 1, _c(P), _c(P), 16, None]),
-    ("gemv misaligned workspace", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 1, _c(P), _c(MIS), 1 << 20, None]),
+    ("gemv batch 0", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 0, _c(P), None]),
+    ("gemv batch 17", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 17, _c(P), None]),
+    ("gemv K%32", "lq_gemv", [_c(P), _c(P), 8, 40, _c(P), 1, _c(P), None]),
+    ("gemv misaligned u", "lq_gemv", [_c(P), _c(P), 8, 64, _c(MIS), 1, _c(P), None]),
+    ("gemv null s", "lq_gemv", [_c(P), None, 8, 64, _c(P), 1, _c(P), None]),
     ("gemm tokens 0", "lq_gemm", [_c(P), _c(P), 8, 64, _c(P), 0, _c(P), None]),
     ("gemm K<32", "lq_gemm", [_c(P), _c(P), 8, 0, _c(P), 4, _c(P), None]),
     ("gemm null o", "lq_gemm", [_c(P), _c(P), 8, 64, _c(P), 4, None, None]),
