@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(256) lift_decode_kernel(LiftArgs p) {
     const int nt = min(DEC_TB, p.batch - t0);
     const int span = r.hi - r.lo;
     float* Ms = smem;                       // [d*D], padded to 16 bytes
-    float* as = Ms + ((p.d * p.D + 3) & ~3); // [span][DEC_TB]
+    float* as = Ms + ((p.d * p.D + 3) & ~3); // [DEC_TB][span]: token-major, so lanes read consecutive channels
     float* aps = as + span * DEC_TB;        // [C][DEC_TB]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(256) lift_decode_kernel(LiftArgs p) {
     for (int i = threadIdx.x; i < p.d * p.D; i += blockDim.x) Ms[i] = __ldg(p.M + i);
     for (int i = threadIdx.x; i < span * nt; i += blockDim.x) {
         int t = i / span, j = i - t * span;
-        as[j * DEC_TB + t] = load_act(p.a, p.a_bf16, (long long)(t0 + t) * p.in + r.lo + j);
+        as[t * span + j] = load_act(p.a, p.a_bf16, (long long)(t0 + t) * p.in + r.lo + j);
     }
     __syncthreads();
 
@@ -162,15 +162,16 @@ __global__ void __launch_bounds__(256) lift_decode_kernel(LiftArgs p) {
                 const int j4 = lane + 32 * q;
                 if (j4 < (p.tblk >> 2)) {
                     const float4 tv = tpre[sl][q];
-                    const float* a0 = as + (base + 4 * j4) * DEC_TB;
+                    const float* a0 = as + base + 4 * j4;  // span and base are multiples of 4 here
 #pragma unroll
                     for (int t = 0; t < DEC_TB; ++t) {
                         if (t < nt) {
+                            const float4 x = *reinterpret_cast<const float4*>(a0 + t * span);
                             float s = acc[t];
-                            s = fmaf(tv.x, a0[t], s);
-                            s = fmaf(tv.y, a0[DEC_TB + t], s);
-                            s = fmaf(tv.z, a0[2 * DEC_TB + t], s);
-                            s = fmaf(tv.w, a0[3 * DEC_TB + t], s);
+                            s = fmaf(tv.x, x.x, s);
+                            s = fmaf(tv.y, x.y, s);
+                            s = fmaf(tv.z, x.z, s);
+                            s = fmaf(tv.w, x.w, s);
                             acc[t] = s;
                         }
                     }
@@ -200,15 +201,16 @@ __global__ void __launch_bounds__(256) lift_decode_kernel(LiftArgs p) {
             if ((p.tblk & 3) == 0) {
                 for (int j4 = lane; j4 < (p.tblk >> 2); j4 += 32) {
                     float4 tv = __ldg(reinterpret_cast<const float4*>(row) + j4);
-                    const float* a0 = as + (base + 4 * j4) * DEC_TB;
+                    const float* a0 = as + base + 4 * j4;
 #pragma unroll
                     for (int t = 0; t < DEC_TB; ++t) {
                         if (t < nt) {
+                            const float4 x = *reinterpret_cast<const float4*>(a0 + t * span);
                             float s = acc[t];
-                            s = fmaf(tv.x, a0[t], s);
-                            s = fmaf(tv.y, a0[DEC_TB + t], s);
-                            s = fmaf(tv.z, a0[2 * DEC_TB + t], s);
-                            s = fmaf(tv.w, a0[3 * DEC_TB + t], s);
+                            s = fmaf(tv.x, x.x, s);
+                            s = fmaf(tv.y, x.y, s);
+                            s = fmaf(tv.z, x.z, s);
+                            s = fmaf(tv.w, x.w, s);
                             acc[t] = s;
                         }
                     }
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(256) lift_decode_kernel(LiftArgs p) {
                     float tv = __ldg(row + j);
 #pragma unroll
                     for (int t = 0; t < DEC_TB; ++t)
-                        if (t < nt) acc[t] = fmaf(tv, as[(base + j) * DEC_TB + t], acc[t]);
+                        if (t < nt) acc[t] = fmaf(tv, as[t * span + base + j], acc[t]);
                 }
             }
 #pragma unroll
@@ -234,7 +236,7 @@ __global__ void __launch_bounds__(256) lift_decode_kernel(LiftArgs p) {
     } else {
         for (int i = threadIdx.x; i < r.C * nt; i += blockDim.x) {
             int ch = i / nt, t = i - ch * nt;
-            aps[ch * DEC_TB + t] = as[ch * DEC_TB + t];
+            aps[ch * DEC_TB + t] = as[t * span + ch];  // span = C, lo = c0 without whitening
         }
     }
     __syncthreads();
