@@ -6,34 +6,43 @@
 //
 // Design (integer tensor-core operands, exact accumulation):
 //   * sum_k sigma u = 2 sum_{bit=1} u - sum_k u, so only the set bits matter.
-//   * Each K-part of u becomes 24-bit fixed point with a per-part, per-column
-//     power-of-two scale (|u_q| <= 2^22: an element's rounding error is at most
-//     2^-22 of the part maximum), held as three balanced int8 digit planes
-//     u_q = d0 + 2^8 d1 + 2^16 d2 -- the bytes of (u_q + 0x808080) ^ 0x808080.
-//     Every CTA quantizes u for itself in its prologue, while its first weight
-//     tiles are in flight; no workspace, no extra launch.
+//   * Each column of u (over the K range of a launch) becomes 24-bit fixed
+//     point with one power-of-two scale (|u_q| < 2^22: an element's rounding
+//     error is at most 2^-22 of the column's largest |u|), held as three
+//     balanced int8 digit planes u_q = d0 + 2^8 d1 + 2^16 d2 -- the bytes of
+//     (u_q + 0x808080) ^ 0x808080. Every CTA quantizes u for itself in its
+//     prologue, one 32-element word per thread: each warp brings its words into
+//     shared memory with TMA (128-byte swizzle, so the per-thread reads are
+//     conflict-free) ahead of its remaining weight prefetch; no workspace, no
+//     extra launch.
 //   * A sign word w yields eight u8 operand registers w & (0x01010101 << j),
 //     j = 0..7: bytes 0 or 2^j for bits j, j+8, j+16, j+24 -- one LOP3 per four
 //     weights, nothing unpacked to memory. These are the A fragments of
 //     mma.sync m16n8k32 u8 x s8 -> s32. (Measured on B200: 0.5 such MMA per
-//     clock per SM = 256 weight bits/clk/SM in isolation, ~155 bits/clk/SM
-//     with the LOP3s and fragment loads of this loop, against ~186 bits/clk/SM
-//     that saturate HBM; tcgen05 kind::i8 with N <= 64 sustains one MMA per ~46
-//     clocks = 90 bits/clk/SM, too slow at decode batch sizes.) B fragments are
-//     the digit planes (MMA column n = 3c + p), read from shared memory where
-//     word x sits at 16-byte chunk 2x + x/4 (a bank skew) with the (j, x),
-//     (j, x+1) digits interleaved, so one conflict-free 16-byte load yields two
-//     aligned B register pairs. One s32 accumulator set per j keeps the 2^j
-//     scales apart; every integer sum is exact.
-//   * About one CTA per SM. A CTA owns G groups of 16 rows; each group's K is
-//     split into H parts, one warp per (group, part), so 12-16 warps keep the
-//     SM busy. Each warp streams its 16 rows through a private ring of 1 KB TMA
-//     tiles (16 rows x 64 bytes: conflict-free fragment reads), one mbarrier
-//     per stage, every wait bounded. The H partial sums of a group are added in
-//     fixed order through shared memory: deterministic results.
+//     clock per SM = 256 weight bits/clk/SM in isolation, against ~186 weight
+//     bits/clk/SM that saturate HBM at 1.97 GHz; the LOP3s load the integer
+//     ALU at the same rate, so the step body carries as little else as
+//     possible. tcgen05 kind::i8 with N <= 64 sustains one MMA per ~46 clocks
+//     = 90 bits/clk/SM, and e4m3 mma.sync runs ~2.6x slower than u8 in this
+//     loop: both too slow at decode batch sizes.) B fragments are the digit
+//     planes (MMA column n = 3c + p), read from shared memory where word pair
+//     (x, x+1), x even, sits in the four 16-byte chunks from 2x + x/4 (a bank
+//     skew), chunk r holding (2r, x), (2r, x+1), (2r+1, x), (2r+1, x+1), so one
+//     conflict-free 16-byte load yields the (adjacent) B register pairs of two
+//     j. One s32 accumulator set per j keeps the 2^j scales apart; every
+//     integer sum is exact.
+//   * One CTA of 12 warps per SM (three per scheduler). A CTA owns a run of
+//     16-row groups; the (group, tile) sequence of its groups is cut into 12
+//     equal contiguous ranges, one per warp, so every scheduler carries the
+//     same load whatever the shape. A tile is two 16-word steps of 16 rows
+//     (2 KB, one 3-D TMA box) when the row length allows, else one step. Each
+//     warp streams its tiles through a private ring, one mbarrier per stage,
+//     every wait bounded. A warp writes one exact partial per group it
+//     touches; the partials of a group are added in warp order: deterministic
+//     results.
 //   * The GEMV is launched as a programmatic dependent of whatever precedes it
-//     on the stream (normally the activation lift): it starts its weight
-//     streams early and waits (griddepcontrol.wait) only before reading u.
+//     on the stream (normally the activation lift): it requests its first
+//     weight tiles early and waits (griddepcontrol.wait) only before reading u.
 //   * Up to two batch columns per pass (six digit planes fill one n8 MMA tile);
 //     larger batches run several passes. K is covered by one launch when the
 //     digit planes fit in shared memory, else by several launches that add into
@@ -50,18 +59,20 @@
 namespace lq {
 namespace {
 
-constexpr int kMaxParts = 8;      // K-parts per row group
-constexpr int kMaxWarps = 16;
+constexpr int kWarps = 12;
+constexpr int kThreads = 32 * kWarps;
 constexpr int kMaxColsPass = 2;   // batch columns per pass (6 digit planes <= n8)
 constexpr int kStepWords = 16;    // words per row a warp consumes per step
-constexpr int kStageBytes = 16 * kStepWords * 4;  // 16 rows x 64 bytes
-constexpr size_t kSmemBudget = 200 * 1024;
+constexpr int kStepBytes = 16 * kStepWords * 4;  // one step of 16 rows x 64 bytes
+constexpr int kMaxRounds = 2;     // quantization items per thread kept in registers (staged path)
+constexpr int kUBoxRows = 16;     // words per TMA box of u
+constexpr size_t kSmemBudget = 220 * 1024;
 
 // Digit-plane storage: 16-byte chunks; word pair (x, x+1), x even, occupies the
-// four chunks from 2x + x/4 holding (j, x), (j, x+1) for j = 0..7 in order.
+// four chunks from 2x + x/4.
 __host__ __device__ __forceinline__ int chunkpos(int x) { return 2 * x + (x >> 2); }
 
-// Chunks per plane for `words` words: covers chunkpos(words - 1) + 1 and is
+// Chunks per plane for `words` words: covers chunkpos(words - 1) + 4 and is
 // 4 (mod 8), which separates the planes a quarter-warp reads.
 __host__ __device__ __forceinline__ int plane_pitch(int words) {
     int cp = 2 * words + words / 4 + 4;
@@ -74,6 +85,23 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
         "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One 16-word step of one 16-row group: words 4t..4t+3 of rows g (ca) and g+8
+// (cb) against this lane's digit chunks bp[0..7].
+__device__ __forceinline__ void mma_step(int (&acc)[8][4], const uint4& ca, const uint4& cb, const uint4* bp) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t a0 = h ? ca.z : ca.x, a2 = h ? ca.w : ca.y;  // row g: words 4t+2h, 4t+2h+1
+        const uint32_t a1 = h ? cb.z : cb.x, a3 = h ? cb.w : cb.y;  // row g+8
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const uint4 b = bp[4 * h + r];  // (2r, x) (2r, x+1) (2r+1, x) (2r+1, x+1)
+            const uint32_t m = 0x01010101u << (2 * r), n = m << 1;
+            mma_u8s8(acc[2 * r], a0 & m, a1 & m, a2 & m, a3 & m, b.x, b.y);
+            mma_u8s8(acc[2 * r + 1], a0 & n, a1 & n, a2 & n, a3 & n, b.z, b.w);
+        }
+    }
 }
 
 __device__ __forceinline__ uint4 load_words(const uint32_t* row, int x, int kw) {
@@ -95,7 +123,7 @@ __device__ __forceinline__ int max_exponent(unsigned cmax_bits) {
     return E == 0 ? -126 : E - 126;
 }
 
-// 32 elements of word x of u (zeros past the end of K).
+// 32 elements of word x of a column of u from global memory (zeros past the end of K).
 __device__ __forceinline__ void load_word(const float* uc, int x, int kw, float (&v)[32]) {
     if (x < kw) {
         const float4* src = reinterpret_cast<const float4*>(uc + 32 * x);
@@ -113,26 +141,48 @@ __device__ __forceinline__ void load_word(const float* uc, int x, int kw, float 
     }
 }
 
+// 32 elements of staged row `row` (128 bytes, 128-byte swizzle: 16-byte chunk q
+// of row r sits at chunk q ^ (r & 7)), or zeros when !valid.
+__device__ __forceinline__ void read_staged(const uint8_t* stage, int row, bool valid, float (&v)[32]) {
+    const uint8_t* base = stage + (size_t)row * 128;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 f = valid ? *reinterpret_cast<const float4*>(base + ((q ^ (row & 7)) << 4))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[4 * q] = f.x;
+        v[4 * q + 1] = f.y;
+        v[4 * q + 2] = f.z;
+        v[4 * q + 3] = f.w;
+    }
+}
+
+// x + 1.5 * 2^23 rounds x to the nearest integer (ties to even) in the low
+// mantissa bits when |x| <= 2^22: the integer is then bits - 0x4B400000.
+constexpr float kRoundMagic = 12582912.0f;
+constexpr uint32_t kMagicBits = 0x4B400000u;
+
 // Digits of one word: P[pl][j] holds, in byte i, digit pl of element j + 8 i.
-__device__ __forceinline__ void word_digits(const float (&v)[32], float sa, float sb, uint32_t (&P)[3][8],
-                                            long long& qsum) {
-    uint32_t tb[32];  // balanced digits of element e in the bytes of tb[e]
+// Returns sum_e u_q[e] (|sum| < 2^27).
+__device__ __forceinline__ int word_digits(const float (&v)[32], float sa, float sb, uint32_t (&P)[3][8]) {
+    uint32_t tb[32];  // balanced digits of element e in bytes 0..2 of tb[e]
+    uint32_t bsum = 0;
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
-        const int qi = __float2int_rn((v[e] * sa) * sb);
-        qsum += qi;
-        tb[e] = (uint32_t)(qi + 0x808080) ^ 0x808080u;
+        const uint32_t b = __float_as_uint(fmaf(v[e] * sa, sb, kRoundMagic));  // u_q = b - kMagicBits
+        bsum += b;
+        tb[e] = (b - (kMagicBits - 0x808080u)) ^ 0x808080u;  // (u_q + 0x808080) ^ 0x808080
     }
 #pragma unroll
-    for (int pl = 0; pl < 3; ++pl) {
-        const uint32_t sel = (uint32_t)pl | ((uint32_t)(pl + 4) << 4);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t lo = __byte_perm(tb[j], tb[j + 8], sel);
-            const uint32_t hi = __byte_perm(tb[j + 16], tb[j + 24], sel);
-            P[pl][j] = __byte_perm(lo, hi, 0x5410);
-        }
+    for (int j = 0; j < 8; ++j) {  // 4x3 byte transpose of elements j, j+8, j+16, j+24
+        const uint32_t t0 = __byte_perm(tb[j], tb[j + 8], 0x5140);        // a0 b0 a1 b1
+        const uint32_t t1 = __byte_perm(tb[j + 16], tb[j + 24], 0x5140);  // c0 d0 c1 d1
+        const uint32_t t2 = __byte_perm(tb[j], tb[j + 8], 0x0062);        // a2 b2 .  .
+        const uint32_t t3 = __byte_perm(tb[j + 16], tb[j + 24], 0x0062);  // c2 d2 .  .
+        P[0][j] = __byte_perm(t0, t1, 0x5410);
+        P[1][j] = __byte_perm(t0, t1, 0x7632);
+        P[2][j] = __byte_perm(t2, t3, 0x5410);
     }
+    return (int)(bsum - 32u * kMagicBits);
 }
 
 struct GemvArgs {
@@ -144,272 +194,350 @@ struct GemvArgs {
     int out, K, kw;
     int c0, ncols;    // columns [c0, c0 + ncols) in this pass (ncols <= 2)
     int kx0, kwc;     // words [kx0, kx0 + kwc) of K in this launch; kx0, kwc multiples of 16
-    int G, H, kp;     // row groups per CTA, K-parts per group, words per part (multiple of 16)
+    int ngroups;      // 16-row groups of the layer; CTA b owns [b*ngroups/grid, (b+1)*ngroups/grid)
+    int maxseg;       // partial-sum slots per warp
     int pitch;        // chunks per shared-memory digit plane
     int accumulate;   // 1: o += this launch's result
 };
 
-__host__ __device__ inline size_t gemv_smem(int G, int H, int ncols, int stages, int pitch, bool tma) {
-    const int W = G * H;
-    size_t s = tma ? (size_t)W * stages * (kStageBytes + 8) : 0;  // rings + their barriers
-    s += (size_t)3 * ncols * pitch * 16 + 128;                     // digit planes + zero block
-    s += (size_t)W * ncols * 16 * 8;                               // partial sums
-    s += (size_t)kMaxColsPass * kMaxParts * (4 + 8);               // per (column, part) max and sum of u_q
-    return s + 16;
+// Shared-memory carve-up (offsets from a 1024-byte-aligned base).
+struct Layout {
+    size_t ring, work, zero, bars, part, sall, colmax, wbound, total;
+};
+
+__host__ __device__ inline Layout gemv_layout(int ts, int stages, bool tma, bool ustage, int ncols, int kwc,
+                                              int pitch, int maxseg) {
+    Layout L;
+    L.ring = 0;
+    const size_t rings = tma ? (size_t)kWarps * stages * ts * kStepBytes : 0;
+    L.work = rings;  // staged u (until quantized), then the digit planes
+    const size_t planes = (size_t)3 * ncols * pitch * 16;
+    const size_t staged = ustage ? (size_t)ncols * kwc * 128 : 0;
+    L.zero = L.work + (((planes > staged ? planes : staged) + 127) & ~(size_t)127);
+    L.bars = L.zero + 128;
+    L.part = L.bars + (size_t)kWarps * (stages + 1) * 8;
+    L.sall = L.part + (size_t)kWarps * maxseg * ncols * 16 * 8;
+    L.colmax = L.sall + kMaxColsPass * 8;
+    L.wbound = L.colmax + kMaxColsPass * 4;
+    L.total = L.wbound + (kWarps + 1) * 4 + 1024;  // + alignment slack
+    return L;
 }
 
-template <int STAGES, bool TMA>
-__global__ void __launch_bounds__(512, 1) gemv_kernel(const __grid_constant__ CUtensorMap tmap, const GemvArgs p) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int W = p.G * p.H;
-    const int nthreads = 32 * W;
+// Digits of word xl of column c into the shared planes: chunk r of the pair
+// holds 32-bit words (2r, x), (2r, x+1), (2r+1, x), (2r+1, x+1).
+__device__ __forceinline__ void store_digits(uint4* planes, int pitch, int c, int xl, const uint32_t (&P)[3][8]) {
+    uint32_t* base = reinterpret_cast<uint32_t*>(planes + chunkpos(xl & ~1)) + (xl & 1);
+#pragma unroll
+    for (int pl = 0; pl < 3; ++pl) {
+        uint32_t* d = base + (size_t)(3 * c + pl) * pitch * 4;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            d[4 * r] = P[pl][2 * r];
+            d[4 * r + 2] = P[pl][2 * r + 1];
+        }
+    }
+}
+
+// Per-column max of |u| (as float bits) into colmax: one shared atomic per warp
+// when the warp's items share a column.
+__device__ __forceinline__ void reduce_max(unsigned* colmax, bool live, int c, unsigned bits, int lane) {
+    const int c_first = __shfl_sync(0xffffffffu, c, 0);
+    if (__all_sync(0xffffffffu, !live || c == c_first)) {
+        const unsigned m = __reduce_max_sync(0xffffffffu, bits);
+        if (lane == 0) atomicMax(colmax + c_first, m);
+    } else if (live) {
+        atomicMax(colmax + c, bits);
+    }
+}
+
+// Per-column sum of u_q (|item sum| < 2^27): split into 16-bit halves so the
+// 32-bit warp reductions cannot overflow.
+__device__ __forceinline__ void reduce_sum(unsigned long long* sall, bool live, int c, int qsum, int lane) {
+    const int c_first = __shfl_sync(0xffffffffu, c, 0);
+    if (__all_sync(0xffffffffu, !live || c == c_first)) {
+        const unsigned lo = __reduce_add_sync(0xffffffffu, (unsigned)(qsum & 0xffff));
+        const int hi = (int)__reduce_add_sync(0xffffffffu, (unsigned)(qsum >> 16));
+        if (lane == 0) atomicAdd(sall + c_first, (unsigned long long)(((long long)hi << 16) + (long long)lo));
+    } else if (live) {
+        atomicAdd(sall + c, (unsigned long long)(long long)qsum);
+    }
+}
+
+__device__ __forceinline__ float absmax32(const float (&v)[32]) {
+    float mx = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, fabsf(v[e]));
+    return mx;
+}
+
+// TS: steps per ring tile (2 with the 3-D weight map, else 1); STAGES: ring
+// depth; TMA: weights through the rings (else guarded register loads); USTAGE:
+// u staged in shared memory by TMA (at most kMaxRounds items per thread).
+template <int TS, int STAGES, bool TMA, bool USTAGE>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap umap, const GemvArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int gi = warp / p.H, h = warp - gi * p.H;
-    const int m0 = blockIdx.x * 16 * p.G;
-    const int wrow0 = m0 + 16 * gi;
-    const int xl_begin = h * p.kp;                                    // local word of this warp's part
-    const int x_begin = p.kx0 + xl_begin;                             // global word
-    const int x_end = min(min(p.kw, p.kx0 + p.kwc), x_begin + p.kp);
-    const int steps = max(0, x_end - x_begin + kStepWords - 1) / kStepWords;
+    const int gbeg = (int)((long long)blockIdx.x * p.ngroups / gridDim.x);
+    const int gend = (int)((long long)(blockIdx.x + 1) * p.ngroups / gridDim.x);
+    const int m0 = 16 * gbeg;
+    const int spg = p.kwc / kStepWords;              // steps per group
+    const int tpg = (spg + TS - 1) / TS;             // tiles per group
+    const int total = (gend - gbeg) * tpg;           // tiles of this CTA
+    const int t0 = (int)((long long)warp * total / kWarps);
+    const int t1 = (int)((long long)(warp + 1) * total / kWarps);
     const int ndig = 3 * p.ncols;
+    constexpr int kTileBytes = TS * kStepBytes;
 
-    uint8_t* ring = smem + (size_t)warp * STAGES * kStageBytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (TMA ? (size_t)W * STAGES * kStageBytes : 0)) + warp * STAGES;
-    uint4* bplanes = reinterpret_cast<uint4*>(smem + (TMA ? (size_t)W * STAGES * (kStageBytes + 8) : 0));
-    uint4* bzero = bplanes + (size_t)ndig * p.pitch;  // 8 zero chunks: digits of idle MMA columns
-    double* part = reinterpret_cast<double*>(bzero + 8);
-    unsigned* colmax = reinterpret_cast<unsigned*>(part + (size_t)W * p.ncols * 16);       // [c][h]
-    unsigned long long* sall = reinterpret_cast<unsigned long long*>(colmax + kMaxColsPass * kMaxParts);
+    const Layout L = gemv_layout(TS, STAGES, TMA, USTAGE, p.ncols, p.kwc, p.pitch, p.maxseg);
+    uint8_t* ring = smem + L.ring + (size_t)warp * STAGES * kTileBytes;
+    uint8_t* work = smem + L.work;
+    uint4* bplanes = reinterpret_cast<uint4*>(work);
+    uint4* bzero = reinterpret_cast<uint4*>(smem + L.zero);  // 8 zero chunks: digits of idle MMA columns
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars) + warp * (STAGES + 1);  // ring stages, then u
+    double* part = reinterpret_cast<double*>(smem + L.part);  // [warp][segment][column][16 rows]
+    unsigned long long* sall = reinterpret_cast<unsigned long long*>(smem + L.sall);
+    unsigned* colmax = reinterpret_cast<unsigned*>(smem + L.colmax);
+    int* wbound = reinterpret_cast<int*>(smem + L.wbound);  // warp w owns tiles [wbound[w], wbound[w+1])
+    const uint32_t ubar = sm100::smem_addr(bars + STAGES);
 
-    if (TMA && lane == 0)
-        for (int st = 0; st < STAGES; ++st) sm100::mbar_init(sm100::smem_addr(bars + st), 1);
-    if (TMA) sm100::fence_barrier_init();
+    // Next tile to request (lane 0): ring index nxt, step xs of its group, row y.
+    int nxt = t0, nxt_xs = 0, nxt_y = 0;
+    if (TMA) {
+        const int gl = t0 / tpg;
+        nxt_xs = (t0 - gl * tpg) * TS;
+        nxt_y = m0 + 16 * gl;
+    }
+    auto issue = [&]() {
+        const int slot = (nxt - t0) & (STAGES - 1);
+        const uint32_t bar = sm100::smem_addr(bars + slot);
+        const uint32_t dst = sm100::smem_addr(ring + slot * kTileBytes);
+        sm100::mbar_arrive_expect_tx(bar, kTileBytes);
+        if (TS == 2)
+            sm100::tma_load_3d(dst, &wmap, 0, nxt_y, p.kx0 / kStepWords + nxt_xs, bar);
+        else
+            sm100::tma_load_2d(dst, &wmap, p.kx0 + nxt_xs * kStepWords, nxt_y, bar);
+        ++nxt;
+        nxt_xs += TS;
+        if (nxt_xs >= spg) {
+            nxt_xs = 0;
+            nxt_y += 16;
+        }
+    };
+    // One tile (two for shallow rings of 1-step tiles) is requested before the
+    // dependency wait, overlapping the kernel before this one; the rest only
+    // after this warp's requests for u, so that those latency-critical loads do
+    // not queue behind ~100 KB of weights per SM.
+    constexpr int kEarly = TS == 1 && STAGES > 4 ? 2 : 1;
+    if (lane == 0) {
+        if (TMA) sm100::prefetch_tensormap(&wmap);
+        if (USTAGE) sm100::prefetch_tensormap(&umap);
+        if (TMA || USTAGE) {
+            for (int st = 0; st <= STAGES; ++st) sm100::mbar_init(sm100::smem_addr(bars + st), 1);
+            sm100::fence_barrier_init();
+        }
+        if (TMA)
+            while (nxt < t1 && nxt < t0 + kEarly) issue();
+    }
     if (threadIdx.x < 8) bzero[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
-    if (threadIdx.x < kMaxColsPass * kMaxParts) {
+    if (threadIdx.x < kMaxColsPass) {
         colmax[threadIdx.x] = 0u;
         sall[threadIdx.x] = 0ull;
     }
+    if (threadIdx.x <= kWarps) wbound[threadIdx.x] = (int)((long long)threadIdx.x * total / kWarps);
     __syncthreads();
-
-    auto issue = [&](int w) {  // lane 0 only
-        const int slot = w & (STAGES - 1);
-        sm100::mbar_arrive_expect_tx(sm100::smem_addr(bars + slot), kStageBytes);
-        sm100::tma_load_2d(sm100::smem_addr(ring + slot * kStageBytes), &tmap, x_begin + w * kStepWords, wrow0,
-                           sm100::smem_addr(bars + slot));
-    };
-    int issued = 0;
-    if (TMA && lane == 0)
-        for (; issued < STAGES - 1 && issued < steps; ++issued) issue(issued);
-
-    const int r0 = wrow0 + g, r1 = r0 + 8;
-    const bool v0 = r0 < p.out, v1 = r1 < p.out;
-    const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
-    const uint32_t* row0 = p.packed + (long long)min(r0, p.out - 1) * p.kw;
-    const uint32_t* row1 = p.packed + (long long)min(r1, p.out - 1) * p.kw;
-    uint4 wa = zero4, wb = zero4;
-    if (!TMA) {
-        wa = v0 ? load_words(row0, x_begin + 4 * t, p.kw) : zero4;
-        wb = v1 ? load_words(row1, x_begin + 4 * t, p.kw) : zero4;
-    }
 
     // u is written by the kernel before this one on the stream
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // ---- quantize this launch's slice of u: item = (column, word pair), key = c * H + part;
-    // pass 1 takes the per-(column, part) maxima, pass 2 writes the digit planes
-    const int npairs = p.kwc / 2;
-    const int nitems = p.ncols * npairs;
-    const int items_round = (nitems + nthreads - 1) / nthreads * nthreads;  // uniform trip count
-    for (int it = threadIdx.x; it < items_round; it += nthreads) {
-        const bool live = it < nitems;
-        const int c = live ? it / npairs : 0, pr = it - c * npairs;
-        const int xg = p.kx0 + 2 * pr;
-        const float* uc = p.u + (long long)(p.c0 + c) * p.K;
-        float a[32], b[32];
-        load_word(uc, live ? xg : p.kw, p.kw, a);
-        load_word(uc, live ? xg + 1 : p.kw, p.kw, b);
-        float mx = 0.f;
+    // ---- quantize this launch's slice of u: item it = (column, word), item
+    // rd * kThreads + threadIdx.x in round rd; pass 1 takes the per-column
+    // maxima, pass 2 writes the digit planes
+    const int nitems = p.ncols * p.kwc;
+    const int nrounds = (nitems + kThreads - 1) / kThreads;
+    float v[kMaxRounds][32];
+    bool ufail = false;
+    if constexpr (USTAGE) {
+        // this warp's items of every round, 16 words per box, staged at row = item
+        if (lane == 0) {
+            uint32_t bytes = 0;
+            for (int rd = 0; rd < nrounds; ++rd)
+                for (int h = 0; h < 2; ++h)
+                    if (rd * kThreads + 32 * warp + kUBoxRows * h < nitems) bytes += kUBoxRows * 128;
+            if (bytes) {
+                sm100::mbar_arrive_expect_tx(ubar, bytes);
+                for (int rd = 0; rd < nrounds; ++rd)
+                    for (int h = 0; h < 2; ++h) {
+                        const int base = rd * kThreads + 32 * warp + kUBoxRows * h;
+                        if (base >= nitems) continue;
+                        const int c = base / p.kwc;
+                        sm100::tma_load_2d(sm100::smem_addr(work + (size_t)base * 128), &umap, 0,
+                                           (p.c0 + c) * p.kw + p.kx0 + (base - c * p.kwc), ubar);
+                    }
+            } else {
+                sm100::mbar_arrive(ubar);
+            }
+            if (TMA)
+                while (nxt < t1 && nxt < t0 + STAGES - 1) issue();
+        }
+        ufail = !sm100::mbar_wait(ubar, 0, p.status);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, fmaxf(fabsf(a[e]), fabsf(b[e])));
-        const unsigned key = live ? (unsigned)(c * p.H + (2 * pr) / p.kp) : 0xffffffffu;
-        const unsigned peers = __match_any_sync(0xffffffffu, key);
-        const unsigned gmax = __reduce_max_sync(peers, __float_as_uint(mx));  // non-negative: bits order like values
-        if (live && lane == __ffs(peers) - 1) atomicMax(colmax + key, gmax);
-    }
-    __syncthreads();
-    for (int it = threadIdx.x; it < items_round; it += nthreads) {
-        const bool live = it < nitems;
-        const int c = live ? it / npairs : 0, pr = it - c * npairs;
-        const int xg = p.kx0 + 2 * pr;
-        const unsigned key = live ? (unsigned)(c * p.H + (2 * pr) / p.kp) : 0xffffffffu;
-        long long qsum = 0;
-        if (live) {
-            const int F = 22 - max_exponent(colmax[key]);  // part max * 2^F < 2^22
-            const float sa = pow2f(F >> 1), sb = pow2f(F - (F >> 1));
-            uint32_t P0[3][8], P1[3][8];
-            const float* uc = p.u + (long long)(p.c0 + c) * p.K;  // second read: L1 hits
-            float a[32];
-            load_word(uc, xg, p.kw, a);
-            word_digits(a, sa, sb, P0, qsum);
-            load_word(uc, xg + 1, p.kw, a);
-            word_digits(a, sa, sb, P1, qsum);
-#pragma unroll
-            for (int pl = 0; pl < 3; ++pl) {
-                uint4* dst = bplanes + (size_t)(3 * c + pl) * p.pitch + chunkpos(2 * pr);
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-                    dst[r] = make_uint4(P0[pl][2 * r], P1[pl][2 * r], P0[pl][2 * r + 1], P1[pl][2 * r + 1]);
+        for (int rd = 0; rd < kMaxRounds; ++rd) {
+            if (rd < nrounds) {
+                const int it = rd * kThreads + threadIdx.x;
+                const bool live = it < nitems;
+                const int c = live ? it / p.kwc : 0;
+                read_staged(work, it, live && p.kx0 + it - c * p.kwc < p.kw, v[rd]);
+                reduce_max(colmax, live, c, __float_as_uint(absmax32(v[rd])), lane);
             }
         }
-        // group sums of u_q (|item sum| < 2^29): split into 16-bit halves so the
-        // 32-bit warp reductions cannot overflow
-        const unsigned peers = __match_any_sync(0xffffffffu, key);
-        const unsigned lo = __reduce_add_sync(peers, (unsigned)(qsum & 0xffff));
-        const int hi = (int)__reduce_add_sync(peers, (unsigned)(int)(qsum >> 16));
-        if (live && lane == __ffs(peers) - 1)
-            atomicAdd(sall + key, (unsigned long long)(((long long)hi << 16) + (long long)lo));
-    }
-    __syncthreads();
-
-    int acc[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[j][e] = 0;
-
-    auto mma_half = [&](uint32_t lo0, uint32_t hi0, uint32_t lo1, uint32_t hi1, const uint32_t (&B)[16]) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t msk = 0x01010101u << j;
-            mma_u8s8(acc[j], lo0 & msk, lo1 & msk, hi0 & msk, hi1 & msk, B[2 * j], B[2 * j + 1]);
-        }
-    };
-    // B fragments: this lane's digit column (or the zero block), words 4t.. of the
-    // step; the B register pair (b0, b1) of j is (B[2j], B[2j+1]).
-    const bool live_col = g < ndig;
-    const uint4* bsrc = live_col ? bplanes + (size_t)g * p.pitch + chunkpos(xl_begin + 4 * t) : bzero;
-    const int binc = live_col ? 36 : 0;  // chunkpos advances 36 chunks per 16-word step
-    auto fetch_b = [&](int half, uint32_t (&B)[16]) {
-        const uint4* src = bsrc + 4 * half;
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const uint4 v = src[r];
-            B[4 * r + 0] = v.x;
-            B[4 * r + 1] = v.y;
-            B[4 * r + 2] = v.z;
-            B[4 * r + 3] = v.w;
-        }
-        if (half) bsrc += binc;
-    };
-
-    bool ok = true;
-    if (TMA) {
-        // Software-pipelined by half steps: the next half's digits (and, at step
-        // boundaries, the next weight tile) are read before the current half's
-        // LOP3s and MMAs are issued.
-        const uint8_t* ring_lane = ring + g * 64 + t * 16;
-        const uint32_t bar0 = sm100::smem_addr(bars);
-        int slot = 0;
-        uint32_t phase = 0;
-        auto fetch_tile = [&](uint4& ca, uint4& cb) -> bool {
-            const uint32_t bar = bar0 + 8 * slot;
-            if (!sm100::mbar_try_wait(bar, phase) && !sm100::mbar_wait(bar, phase, p.status)) return false;
-            const uint8_t* st = ring_lane + slot * kStageBytes;
-            ca = *reinterpret_cast<const uint4*>(st);
-            cb = *reinterpret_cast<const uint4*>(st + 8 * 64);
-            __syncwarp();  // every lane has read the slot before lane 0 refills it
-            if (lane == 0 && issued < steps) issue(issued++);
-            slot = (slot + 1) & (STAGES - 1);
-            phase ^= slot == 0;
-            return true;
-        };
-        uint4 ca = zero4, cb = zero4;
-        uint32_t Bc[16], Bn[16];
-        if (steps > 0) {
-            ok = fetch_tile(ca, cb);  // flagged in the status word on timeout; results invalid
-            fetch_b(0, Bc);
-        }
-        for (int w = 0; ok && w < steps; ++w) {
-            fetch_b(1, Bn);
-            mma_half(ca.x, ca.y, cb.x, cb.y, Bc);
-            const uint32_t lo0 = ca.z, hi0 = ca.w, lo1 = cb.z, hi1 = cb.w;
-            if (w + 1 < steps) {
-                ok = fetch_tile(ca, cb);
-                fetch_b(0, Bc);
-            }
-            mma_half(lo0, hi0, lo1, hi1, Bn);
-        }
-        // Leave nothing in flight: on the normal path every issued tile was waited
-        // for; after a timeout, wait (bounded) for the rest.
-        if (lane == 0 && !ok)
-            for (int w = issued - (STAGES - 1) < 0 ? 0 : issued - (STAGES - 1); w < issued; ++w)
-                sm100::mbar_wait(sm100::smem_addr(bars + (w & (STAGES - 1))), (w / STAGES) & 1, p.status);
-        __syncwarp();
     } else {
-        for (int w = 0; w < steps; ++w) {
-            const uint4 ca = wa, cb = wb;
-            if (w + 1 < steps) {
-                const int xn = x_begin + (w + 1) * kStepWords + 4 * t;
-                wa = v0 ? load_words(row0, xn, p.kw) : zero4;
-                wb = v1 ? load_words(row1, xn, p.kw) : zero4;
-            }
-            uint32_t B[16];
-            fetch_b(0, B);
-            mma_half(ca.x, ca.y, cb.x, cb.y, B);
-            fetch_b(1, B);
-            mma_half(ca.z, ca.w, cb.z, cb.w, B);
+        for (int rd = 0; rd < nrounds; ++rd) {
+            const int it = rd * kThreads + threadIdx.x;
+            const bool live = it < nitems;
+            const int c = live ? it / p.kwc : 0;
+            load_word(p.u + (long long)(p.c0 + c) * p.K, live ? p.kx0 + it - c * p.kwc : p.kw, p.kw, v[0]);
+            if (TMA && rd == 0 && lane == 0)
+                while (nxt < t1 && nxt < t0 + STAGES - 1) issue();
+            reduce_max(colmax, live, c, __float_as_uint(absmax32(v[0])), lane);
         }
     }
-
-    // ---- combine the eight 2^j accumulators: V = sum_j 2^(7-j) acc_j = 2^7 sum_k bit*d,
-    // then gather the three planes of each column with shuffles
-    double vreg[4];
+    __syncthreads();  // every staged word has been read: the planes may overwrite the staging area
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        long long v = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v += (long long)acc[j][e] * (1ll << (7 - j));
-        vreg[e] = (double)v;
-    }
-    double* out_part = part + (size_t)warp * p.ncols * 16;  // [ncols][16 rows]
-    for (int c = 0; c < p.ncols; ++c) {
-        const int key = c * p.H + h;
-        const int F = 22 - max_exponent(colmax[key]);
-        const double unscale = __longlong_as_double((long long)(1023 - F) << 52);
-        const double sq = (double)(long long)sall[key];
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {  // rows g (hr = 0) and g + 8
-            double s1 = 0.0;
-#pragma unroll
-            for (int pl = 0; pl < 3; ++pl) {
-                const int col = 3 * c + pl, e = 2 * hr + (col & 1);
-                double mine = 0.0;
-#pragma unroll
-                for (int ee = 0; ee < 4; ++ee)
-                    if (ee == e) mine = vreg[ee];
-                const double v = __shfl_sync(0xffffffffu, mine, (lane & ~3) | (col >> 1));
-                s1 += (pl == 0 ? 1.0 : pl == 1 ? 256.0 : 65536.0) * v;  // exact: 2^7 sum_{bit=1} u_q
+    for (int rd = 0; rd < (USTAGE ? kMaxRounds : 1); ++rd) {
+        for (int r2 = rd; r2 < (USTAGE ? rd + 1 : nrounds); ++r2) {
+            if (USTAGE && r2 >= nrounds) break;
+            const int it = r2 * kThreads + threadIdx.x;
+            const bool live = it < nitems;
+            const int c = live ? it / p.kwc : 0;
+            const int xl = it - c * p.kwc;
+            int qsum = 0;
+            if (live) {
+                if (!USTAGE && nrounds > 1) load_word(p.u + (long long)(p.c0 + c) * p.K, p.kx0 + xl, p.kw, v[0]);
+                const int F = 22 - max_exponent(colmax[c]);  // column max * 2^F < 2^22
+                uint32_t P[3][8];
+                qsum = word_digits(v[rd], pow2f(F >> 1), pow2f(F - (F >> 1)), P);
+                store_digits(bplanes, p.pitch, c, xl, P);
             }
-            // sum_k sigma u_q = 2 sum_{bit=1} u_q - sum_k u_q, then undo the 2^F scale
-            if (t == 0) out_part[c * 16 + g + 8 * hr] = (s1 * (1.0 / 64.0) - sq) * unscale;
+            reduce_sum(sall, live, c, qsum, lane);
         }
     }
     __syncthreads();
 
-    // ---- add the H parts of each row group in fixed order, scale, store
-    if (h == 0) {
-        for (int item = lane; item < 16 * p.ncols; item += 32) {
-            const int row = item & 15, c = item >> 4;
-            const int m = wrow0 + row;
-            if (m < p.out) {
-                double sum = 0.0;
-                for (int hh = 0; hh < p.H; ++hh) sum += part[((size_t)(gi * p.H + hh) * p.ncols + c) * 16 + row];
-                float* dst = p.o + (long long)(p.c0 + c) * p.out + m;
-                const float val = (float)(sum * (double)__ldg(p.s + m));
-                *dst = p.accumulate ? *dst + val : val;
+    // ---- main loop: this warp's tiles [t0, t1), one segment per group touched
+    const bool live_col = g < ndig;
+    const uint4* bcol = live_col ? bplanes + (size_t)g * p.pitch + 9 * t : bzero;
+    const int binc = live_col ? 36 : 0;  // chunkpos advances 36 chunks per 16-word step
+    const uint8_t* ring_lane = ring + g * 64 + t * 16;
+    const uint32_t bar0 = sm100::smem_addr(bars);
+    const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+    int kfail = -1;  // ring index whose wait ran out
+    int seg = 0;
+    for (int tt = t0; tt < t1; ++seg) {
+        const int gl = tt / tpg;
+        const int tend = min(t1, (gl + 1) * tpg);
+        int acc[8][4];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[j][e] = 0;
+        int xs = (tt - gl * tpg) * TS;
+        const uint4* bp = bcol + binc * xs;
+        const int r0 = m0 + 16 * gl + g, r1 = r0 + 8;
+        const uint32_t* row0 = p.packed + (long long)min(r0, p.out - 1) * p.kw;
+        const uint32_t* row1 = p.packed + (long long)min(r1, p.out - 1) * p.kw;
+        const bool v0 = r0 < p.out, v1 = r1 < p.out;
+        for (; tt < tend; ++tt, xs += TS) {
+            uint4 ca0, cb0, ca1 = zero4, cb1 = zero4;
+            if (TMA) {
+                const int k = tt - t0;
+                const uint32_t bar = bar0 + 8 * (k & (STAGES - 1));
+                const uint32_t par = (k / STAGES) & 1;
+                if (!sm100::mbar_try_wait(bar, par) && !sm100::mbar_wait(bar, par, p.status)) {
+                    kfail = k;  // flagged in the status word; results invalid
+                    break;
+                }
+                const uint8_t* st = ring_lane + (k & (STAGES - 1)) * kTileBytes;
+                ca0 = *reinterpret_cast<const uint4*>(st);
+                cb0 = *reinterpret_cast<const uint4*>(st + 8 * 64);
+                if (TS == 2) {
+                    ca1 = *reinterpret_cast<const uint4*>(st + kStepBytes);
+                    cb1 = *reinterpret_cast<const uint4*>(st + kStepBytes + 8 * 64);
+                }
+                __syncwarp();  // every lane has read the slot before lane 0 refills the previous one
+                if (lane == 0 && nxt < t1) issue();
+            } else {
+                const int x = p.kx0 + xs * kStepWords + 4 * t;
+                ca0 = v0 ? load_words(row0, x, p.kw) : zero4;
+                cb0 = v1 ? load_words(row1, x, p.kw) : zero4;
+            }
+            mma_step(acc, ca0, cb0, bp);
+            bp += binc;
+            if (TS == 2 && xs + 1 < spg) {
+                mma_step(acc, ca1, cb1, bp);
+                bp += binc;
             }
         }
+        if (kfail >= 0) break;
+        // ---- segment partial: V = sum_j 2^(7-j) acc_j = 2^7 sum_{bit=1} d per digit
+        // column; gather the three planes of each batch column with shuffles
+        double vreg[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            long long vv = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) vv += (long long)acc[j][e] * (1ll << (7 - j));
+            vreg[e] = (double)vv;
+        }
+        double* dst = part + (size_t)(warp * p.maxseg + seg) * p.ncols * 16;
+        for (int c = 0; c < p.ncols; ++c) {
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {  // rows g (hr = 0) and g + 8
+                double s1 = 0.0;
+#pragma unroll
+                for (int pl = 0; pl < 3; ++pl) {
+                    const int col = 3 * c + pl, e = 2 * hr + (col & 1);
+                    double mine = 0.0;
+#pragma unroll
+                    for (int ee = 0; ee < 4; ++ee)
+                        if (ee == e) mine = vreg[ee];
+                    const double vv = __shfl_sync(0xffffffffu, mine, (lane & ~3) | (col >> 1));
+                    s1 += (pl == 0 ? 1.0 : pl == 1 ? 256.0 : 65536.0) * vv;  // exact: 2^7 sum_{bit=1} u_q
+                }
+                if (t == 0) dst[c * 16 + g + 8 * hr] = s1 * (1.0 / 64.0);  // 2 sum_{bit=1} u_q
+            }
+        }
+    }
+    if (lane == 0) {
+        // leave nothing in flight after a wait ran out: wait (bounded) for the
+        // tiles requested from the failed one on, and for u
+        if (TMA && kfail >= 0)
+            for (int k = kfail; k < nxt - t0; ++k)
+                sm100::mbar_wait(bar0 + 8 * (k & (STAGES - 1)), (k / STAGES) & 1, p.status, 100000000ull);
+        if (USTAGE && ufail) sm100::mbar_wait(ubar, 0, p.status, 100000000ull);
+    }
+    __syncthreads();
+
+    // ---- per (group, column, row): add the warps' partials in warp order, finish, store
+    const int nout = (gend - gbeg) * p.ncols * 16;
+    for (int item = threadIdx.x; item < nout; item += kThreads) {
+        const int row = item & 15, c = (item >> 4) % p.ncols, gl = (item >> 4) / p.ncols;
+        const int m = m0 + 16 * gl + row;
+        if (m >= p.out) continue;
+        double sum = 0.0;
+        for (int w = 0; w < kWarps; ++w) {
+            const int a = wbound[w], b = wbound[w + 1];
+            if (a < b && a < (gl + 1) * tpg && b > gl * tpg)  // empty ranges touch no group
+                sum += part[((size_t)(w * p.maxseg + (gl - a / tpg)) * p.ncols + c) * 16 + row];
+        }
+        const int F = 22 - max_exponent(colmax[c]);
+        // sum_k sigma u_q = 2 sum_{bit=1} u_q - sum_k u_q, then undo the 2^F scale
+        const double val = (sum - (double)(long long)sall[c]) * __longlong_as_double((long long)(1023 - F) << 52);
+        float* out = p.o + (long long)(p.c0 + c) * p.out + m;
+        const float res = (float)(val * (double)__ldg(p.s + m));
+        *out = p.accumulate ? *out + res : res;
     }
 }
 
@@ -442,58 +570,89 @@ EncodeTiledFn encode_fn() {
 }
 
 struct Plan {
-    int G, H, kp, stages, cols, kwc, pitch;
-    bool tma;
+    int grid, ts, stages, cols, kwc, pitch, maxseg;
+    bool tma, ustage;
+    size_t smem;
 };
 
-// About one CTA per SM, one warp per (16-row group, K-part); the widest K chunk
-// (and up to two columns) whose digit planes fit in shared memory.
+// Partial-sum slots a warp needs: the groups its tile range can touch.
+int max_segments(int grid, int ngroups, int tpg) {
+    const long long gmax = (ngroups + grid - 1) / grid;
+    const long long len = (gmax * tpg + kWarps - 1) / kWarps;
+    return (int)((len + tpg - 1) / tpg + 1);
+}
+
+// One CTA per SM (or per group when there are fewer groups); the widest K chunk
+// and up to two columns whose digit planes fit in shared memory, preferring a
+// deep ring, then u staged by TMA.
 Plan make_plan(int out, int kw, int batch) {
-    const int sms = num_sms();
-    const int groups = (out + 15) / 16;
+    const int ngroups = (out + 15) / 16;
     const int kwp = (kw + 15) / 16 * 16;
     Plan pl;
     pl.tma = (kw % 4) == 0;
-    pl.G = std::max(1, std::min(kMaxWarps, (groups + sms - 1) / sms));
+    pl.ts = pl.tma && kw % 16 == 0 ? 2 : 1;
+    pl.grid = std::min(num_sms(), ngroups);
     for (int nchunks = 1;; ++nchunks) {
         pl.kwc = ((kwp + nchunks - 1) / nchunks + 15) / 16 * 16;
-        pl.H = std::max(1, std::min(kMaxParts, kMaxWarps / pl.G));
-        pl.H = std::min(pl.H, pl.kwc / kStepWords);  // at least one step per part
-        pl.kp = ((pl.kwc + pl.H - 1) / pl.H + kStepWords - 1) / kStepWords * kStepWords;
-        pl.H = (pl.kwc + pl.kp - 1) / pl.kp;  // drop empty parts
-        pl.stages = pl.G * pl.H <= 8 ? 8 : 4;
         pl.pitch = plane_pitch(pl.kwc);
+        const int tpg = (pl.kwc / kStepWords + pl.ts - 1) / pl.ts;
+        pl.maxseg = max_segments(pl.grid, ngroups, tpg);
         for (int cols = std::min(kMaxColsPass, batch); cols >= 1; --cols) {
             pl.cols = cols;
-            if (gemv_smem(pl.G, pl.H, cols, pl.stages, pl.pitch, pl.tma) <= kSmemBudget) return pl;
+            const int nrounds = (cols * pl.kwc + kThreads - 1) / kThreads;
+            for (int deep = pl.tma ? 1 : 0; deep >= 0; --deep) {
+                pl.stages = (pl.ts == 2 ? 2 : 4) * (deep ? 2 : 1);  // the register path is built for 4
+                for (int us = 1; us >= 0; --us) {
+                    pl.ustage = us && pl.tma && nrounds <= kMaxRounds;
+                    if (us && !pl.ustage) continue;
+                    pl.smem = gemv_layout(pl.ts, pl.stages, pl.tma, pl.ustage, cols, pl.kwc, pl.pitch, pl.maxseg).total;
+                    if (pl.smem <= kSmemBudget) return pl;
+                }
+            }
         }
     }
 }
 
-template <int STAGES, bool TMA>
-cudaError_t launch_kernel(const CUtensorMap& map, const GemvArgs& p, cudaStream_t st) {
-    const size_t smem = gemv_smem(p.G, p.H, p.ncols, STAGES, p.pitch, TMA);
+template <int TS, int STAGES, bool TMA, bool USTAGE>
+cudaError_t launch_kernel(const CUtensorMap& wmap, const CUtensorMap& umap, const GemvArgs& p, const Plan& pl,
+                          cudaStream_t st) {
+    auto kern = gemv_kernel<TS, STAGES, TMA, USTAGE>;
     static size_t granted[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 64 || granted[dev] < smem) {
-        cudaError_t e =
-            cudaFuncSetAttribute(gemv_kernel<STAGES, TMA>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (dev >= 64 || granted[dev] < pl.smem) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
         if (e != cudaSuccess) return e;
-        if (dev < 64) granted[dev] = smem;
+        if (dev < 64) granted[dev] = pl.smem;
     }
-    const int groups = (p.out + 15) / 16;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((groups + p.G - 1) / p.G, 1, 1);
-    cfg.blockDim = dim3(32 * p.G * p.H, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.gridDim = dim3(pl.grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemv_kernel<STAGES, TMA>, map, p);
+    return cudaLaunchKernelEx(&cfg, kern, wmap, umap, p);
+}
+
+cudaError_t launch_planned(const CUtensorMap& wmap, const CUtensorMap& umap, const GemvArgs& p, const Plan& pl,
+                           cudaStream_t st) {
+    if (!pl.tma) return launch_kernel<1, 4, false, false>(wmap, umap, p, pl, st);
+    if (pl.ts == 2) {
+        if (pl.stages == 4)
+            return pl.ustage ? launch_kernel<2, 4, true, true>(wmap, umap, p, pl, st)
+                             : launch_kernel<2, 4, true, false>(wmap, umap, p, pl, st);
+        return pl.ustage ? launch_kernel<2, 2, true, true>(wmap, umap, p, pl, st)
+                         : launch_kernel<2, 2, true, false>(wmap, umap, p, pl, st);
+    }
+    if (pl.stages == 8)
+        return pl.ustage ? launch_kernel<1, 8, true, true>(wmap, umap, p, pl, st)
+                         : launch_kernel<1, 8, true, false>(wmap, umap, p, pl, st);
+    return pl.ustage ? launch_kernel<1, 4, true, true>(wmap, umap, p, pl, st)
+                     : launch_kernel<1, 4, true, false>(wmap, umap, p, pl, st);
 }
 
 }  // namespace
@@ -503,19 +662,41 @@ cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, 
     const int kw = K / 32;
     const Plan pl = make_plan(out, kw, batch);
 
-    CUtensorMap map;
-    memset(&map, 0, sizeof(map));
-    if (pl.tma) {
+    CUtensorMap wmap, umap;
+    memset(&wmap, 0, sizeof(wmap));
+    memset(&umap, 0, sizeof(umap));
+    if (pl.tma || pl.ustage) {
         EncodeTiledFn encode = encode_fn();
         if (!encode) return cudaErrorNotSupported;
-        cuuint64_t gdim[2] = {(cuuint64_t)kw, (cuuint64_t)out};
-        cuuint64_t gstride[1] = {(cuuint64_t)kw * 4};
-        cuuint32_t box[2] = {kStepWords, 16};
-        cuuint32_t estride[2] = {1, 1};
-        if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(packed), gdim, gstride, box, estride,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
+        if (pl.ts == 2) {  // [chunk of 16 words][row][word in chunk]: one box = two steps of 16 rows
+            cuuint64_t gdim[3] = {(cuuint64_t)kStepWords, (cuuint64_t)out, (cuuint64_t)(kw / kStepWords)};
+            cuuint64_t gstride[2] = {(cuuint64_t)kw * 4, (cuuint64_t)kStepWords * 4};
+            cuuint32_t box[3] = {kStepWords, 16, 2};
+            cuuint32_t estride[3] = {1, 1, 1};
+            if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(packed), gdim, gstride, box,
+                       estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        } else if (pl.tma) {
+            cuuint64_t gdim[2] = {(cuuint64_t)kw, (cuuint64_t)out};
+            cuuint64_t gstride[1] = {(cuuint64_t)kw * 4};
+            cuuint32_t box[2] = {kStepWords, 16};
+            cuuint32_t estride[2] = {1, 1};
+            if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(packed), gdim, gstride, box,
+                       estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
+        if (pl.ustage) {  // u as rows of one word (32 floats, 128 bytes)
+            cuuint64_t gdim[2] = {32, (cuuint64_t)batch * kw};
+            cuuint64_t gstride[1] = {128};
+            cuuint32_t box[2] = {32, kUBoxRows};
+            cuuint32_t estride[2] = {1, 1};
+            if (encode(&umap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(u), gdim, gstride, box, estride,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
     }
     for (int c0 = 0; c0 < batch; c0 += pl.cols) {
         for (int kx0 = 0; kx0 < kw; kx0 += pl.kwc) {
@@ -532,14 +713,11 @@ cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, 
             p.ncols = std::min(pl.cols, batch - c0);
             p.kx0 = kx0;
             p.kwc = pl.kwc;
-            p.G = pl.G;
-            p.H = pl.H;
-            p.kp = pl.kp;
+            p.ngroups = (out + 15) / 16;
+            p.maxseg = pl.maxseg;
             p.pitch = pl.pitch;
             p.accumulate = kx0 > 0;
-            cudaError_t e = !pl.tma ? launch_kernel<4, false>(map, p, st)
-                            : pl.stages == 8 ? launch_kernel<8, true>(map, p, st)
-                                             : launch_kernel<4, true>(map, p, st);
+            cudaError_t e = launch_planned(wmap, umap, p, pl, st);
             if (e != cudaSuccess) return e;
         }
     }
