@@ -111,6 +111,34 @@ def test_lift_padding_and_small_blocks(lq):
         assert rel_err(u, want) <= 1e-6
 
 
+@pytest.mark.parametrize("in_dim,d,D,tblk,batch,a_bf16,u_dtype", [
+    (1024, 16, 48, 256, 3, True, "f32"),   # two float4 per lane of a T row, second M column per lane
+    (960, 10, 40, 96, 2, False, "f32"),    # d-blocks straddling whitening blocks
+    (600, 5, 9, 20, 16, True, "f32"),      # narrow blocks, full decode batch, padded lifted tail
+    (600, 5, 9, 20, 2, True, "bf16"),      # bf16 lifted output from the decode path
+    (512, 16, 64, 0, 4, False, "f32"),     # T = identity
+    (1280, 20, 40, 128, 2, True, "f32"),   # d > 16: the shared-memory decode kernel
+])
+def test_lift_decode_shapes(lq, in_dim, d, D, tblk, batch, a_bf16, u_dtype):
+    from datagen.inputs import bf16_bits_from_f32
+    g = rng_for(61, in_dim, d * 1000 + batch)
+    a32 = g.standard_normal((batch, in_dim)).astype(np.float32)
+    a = bf16_bits_from_f32(a32) if a_bf16 else a32
+    M = (g.standard_normal((d, D)) / np.sqrt(D)).astype(np.float32)
+    tinv = (g.standard_normal((in_dim // tblk, tblk, tblk)) / np.sqrt(tblk)).astype(np.float32) if tblk else None
+    K = oracle.lifted_dim(in_dim, d, D)
+    u = host(lq.lift_activations(dev(a), dev(M), K, tinv=None if tinv is None else dev(tinv), u_dtype=u_dtype))
+    want = oracle.lift(oracle.whiten(oracle.to_f64(a, "bf16" if a_bf16 else "f32"),
+                                     None if tinv is None else oracle.to_f64(tinv)), oracle.to_f64(M), K)
+    kreal = (in_dim // d) * D
+    if u_dtype == "bf16":
+        u = oracle.to_f64(u, "bf16")
+        assert np.all(np.abs(u - want) <= _bf16_ulp(want) + 1e-6 * np.max(np.abs(want)))
+    else:
+        assert rel_err(u, want) <= 1e-6
+    assert np.all(u[:, kreal:] == 0.0)
+
+
 # ------------------------------------------------------------------ decode GEMV
 
 @pytest.mark.parametrize("batch", [1, 4])
