@@ -57,7 +57,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const float* __restrict__ s, int out, int K, int tokens, float* __restrict__ o,
                 unsigned* status) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned for the 128-byte swizzle; offsetting the array itself
+    // keeps derived pointers in the shared address space
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES * A_STAGE;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);

@@ -277,7 +277,9 @@ template <int TS, int STAGES, bool TMA, bool USTAGE>
 __global__ void __launch_bounds__(kThreads, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap umap, const GemvArgs p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned (the 128-byte swizzle of staged u); offsetting the array
+    // itself keeps every derived pointer in the shared address space
+    uint8_t* smem = smem_raw + ((1024u - (sm100::smem_addr(smem_raw) & 1023u)) & 1023u);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int gbeg = (int)((long long)blockIdx.x * p.ngroups / gridDim.x);
