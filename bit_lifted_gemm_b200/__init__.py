@@ -23,7 +23,7 @@ LQ_OK, LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_TIMEOUT = 0, 
 LQ_F32, LQ_BF16 = 0, 1
 
 SYMBOLS = ("lq_status_str", "lq_lifted_dim", "lq_pack_signs", "lq_unpack_signs", "lq_lift_activations",
-           "lq_gemv", "lq_gemm", "lq_get_device_status")
+           "lq_gemv", "lq_lift_gemv", "lq_gemm", "lq_get_device_status")
 
 
 class LQError(RuntimeError):
@@ -49,6 +49,8 @@ def _load() -> ctypes.CDLL:
     lib.lq_lift_activations.argtypes = [p, i, i, i, p, i, p, i, i, p, i, i, p]
     lib.lq_gemv.restype = i
     lib.lq_gemv.argtypes = [p, p, i, i, p, i, p, p]
+    lib.lq_lift_gemv.restype = i
+    lib.lq_lift_gemv.argtypes = [p, i, i, i, p, i, p, i, i, p, p, i, i, p, p, p]
     lib.lq_gemm.restype = i
     lib.lq_gemm.argtypes = [p, p, i, i, p, i, p, p]
     lib.lq_get_device_status.restype = i
@@ -141,6 +143,28 @@ def gemv(packed, s, u, out=None, stream=None):
         out = torch.empty((batch, rows), dtype=torch.float32, device=u.device)
     _check(lib.lq_gemv(_ptr(packed), _ptr(s), rows, K, _ptr(u), batch, _ptr(out), _stream(stream)), "lq_gemv")
     return out
+
+
+def lift_gemv(a, M, packed, s, K, tinv=None, u=None, out=None, stream=None):
+    """Fused decode step: a [batch][in] (float32 or bfloat16) -> (u fp32 [batch][K], o fp32 [batch][out])."""
+    import torch
+    _dev_tensor(a, "a")
+    _dev_tensor(M, "M")
+    _dev_tensor(packed, "packed")
+    batch, in_dim = a.shape
+    d, D = M.shape
+    rows = packed.shape[0]
+    a_t = LQ_BF16 if a.dtype == torch.bfloat16 else LQ_F32
+    if u is None:
+        u = torch.empty((batch, K), dtype=torch.float32, device=a.device)
+    if out is None:
+        out = torch.empty((batch, rows), dtype=torch.float32, device=a.device)
+    tblk = 0 if tinv is None else int(tinv.shape[-1])
+    if tinv is not None:
+        _dev_tensor(tinv, "tinv")
+    _check(lib.lq_lift_gemv(_ptr(a), a_t, batch, in_dim, _ptr(tinv), tblk, _ptr(M), d, D, _ptr(packed), _ptr(s),
+                            rows, K, _ptr(u), _ptr(out), _stream(stream)), "lq_lift_gemv")
+    return u, out
 
 
 def gemm(packed, s, u, out=None, stream=None):

@@ -116,6 +116,28 @@ int lq_gemv(const uint32_t* packed, const float* s, int out, int K, const float*
     return from_cuda(lq::launch_gemv(packed, s, out, K, u, batch, o, status, static_cast<cudaStream_t>(stream)));
 }
 
+int lq_lift_gemv(const void* a, int a_dtype, int batch, int in, const float* tinv, int tblk, const float* M, int d,
+                 int D, const uint32_t* packed, const float* s, int out, int K, float* u, float* o, void* stream) {
+    if (!a || !M || !u || !packed || !s || !o) return LQ_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(M) || !aligned16(u) || !aligned16(packed) || !aligned16(s) || !aligned16(o))
+        return LQ_ERR_INVALID_ARG;
+    if (tinv && !aligned16(tinv)) return LQ_ERR_INVALID_ARG;
+    if (a_dtype != LQ_F32 && a_dtype != LQ_BF16) return LQ_ERR_INVALID_ARG;
+    if (batch < 1 || batch > 16 || in < 1 || d < 1 || d > 64 || D < 1 || D > 256 || d * D > 4096)
+        return LQ_ERR_INVALID_ARG;
+    if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
+    if (tinv && (tblk < 1 || tblk > 256 || in % tblk != 0)) return LQ_ERR_INVALID_ARG;
+    if (out < 1) return LQ_ERR_INVALID_ARG;
+    const int sm = is_sm100();
+    if (sm < 0) return LQ_ERR_CUDA;
+    if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    int err = LQ_OK;
+    unsigned* status = status_word(&err);
+    if (!status) return err;
+    return from_cuda(lq::launch_lift_gemv(a, a_dtype == LQ_BF16, batch, in, tinv, tblk, M, d, D, packed, s, out, K, u,
+                                          o, status, static_cast<cudaStream_t>(stream)));
+}
+
 int lq_gemm(const uint32_t* packed, const float* s, int out, int K, const uint16_t* u_bf16, int tokens, float* o,
             void* stream) {
     if (!packed || !s || !u_bf16 || !o) return LQ_ERR_INVALID_ARG;

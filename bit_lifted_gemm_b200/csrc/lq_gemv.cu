@@ -274,7 +274,7 @@ __device__ __forceinline__ float absmax32(const float (&v)[32]) {
 // depth; TMA: weights through the rings (else guarded register loads); USTAGE:
 // u staged in shared memory by TMA (at most kMaxRounds items per thread).
 template <int TS, int STAGES, bool TMA, bool USTAGE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift beside it
     gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap umap, const GemvArgs p) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned (the 128-byte swizzle of staged u); offsetting the array
@@ -724,6 +724,14 @@ cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, 
         }
     }
     return cudaGetLastError();
+}
+
+cudaError_t launch_lift_gemv(const void* a, bool a_bf16, int batch, int in, const float* tinv, int tblk,
+                             const float* M, int d, int D, const uint32_t* packed, const float* s, int out, int K,
+                             float* u, float* o, unsigned* status, cudaStream_t st) {
+    cudaError_t e = launch_lift(a, a_bf16, batch, in, tinv, tblk, M, d, D, u, false, K, st);
+    if (e != cudaSuccess) return e;
+    return launch_gemv(packed, s, out, K, u, batch, o, status, st);  // a programmatic dependent of the lift
 }
 
 }  // namespace lq

@@ -23,6 +23,12 @@ cudaError_t launch_lift(const void* a, bool a_bf16, int batch, int in, const flo
 cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u,
                         int batch, float* o, unsigned* status, cudaStream_t st);
 
+// Decode step: the lift into u, then the GEMV (a programmatic dependent of the
+// lift, so its prologue overlaps the lift where both fit on an SM).
+cudaError_t launch_lift_gemv(const void* a, bool a_bf16, int batch, int in, const float* tinv, int tblk,
+                             const float* M, int d, int D, const uint32_t* packed, const float* s, int out, int K,
+                             float* u, float* o, unsigned* status, cudaStream_t st);
+
 // Prefill GEMM on tcgen05. `status` is the device status word.
 cudaError_t launch_gemm(const uint32_t* packed, const float* s, int out, int K,
                         const uint16_t* u_bf16, int tokens, float* o, unsigned* status,

@@ -98,6 +98,20 @@ LQ_API int lq_lift_activations(const void* a, int a_dtype, int batch, int in,
 LQ_API int lq_gemv(const uint32_t* packed, const float* s, int out, int K,
             const float* u, int batch, float* o, void* stream);
 
+/* Decode step in one call: lq_lift_activations followed by lq_gemv (the small
+ * matmul T* a, then the 1-bit x float matmul and diag(s) -- "Key designs" 4),
+ * with the arguments of both calls:
+ *   a, a_dtype, batch, in, tinv, tblk, M, d, D, K : as lq_lift_activations
+ *   packed, s, out                               : as lq_gemv
+ *   u : fp32 [batch][K] (written: the lifted activations)
+ *   o : fp32 [batch][out] (written); 1 <= batch <= 16
+ * Results are exactly those of the two calls; the GEMV is launched as a
+ * programmatic dependent of the lift, so its setup and first weight requests
+ * overlap the lift. Requires an sm_100 device (else LQ_ERR_UNSUPPORTED). */
+LQ_API int lq_lift_gemv(const void* a, int a_dtype, int batch, int in, const float* tinv, int tblk,
+                        const float* M, int d, int D, const uint32_t* packed, const float* s, int out, int K,
+                        float* u, float* o, void* stream);
+
 /* Prefill 1-bit GEMM on the tensor cores (tcgen05, bf16 operands, fp32 accumulate):
  *   o[t][r] = s[r] * sum_k sigma[r][k] * u[t][k]
  *   packed : uint32 [out][K/32]; s : fp32 [out]; u_bf16 : bf16 bits [tokens][K]

@@ -66,6 +66,16 @@ def _c(v):
     ("gemv K%32", "lq_gemv", [_c(P), _c(P), 8, 40, _c(P), 1, _c(P), None]),
     ("gemv misaligned u", "lq_gemv", [_c(P), _c(P), 8, 64, _c(MIS), 1, _c(P), None]),
     ("gemv null s", "lq_gemv", [_c(P), None, 8, 64, _c(P), 1, _c(P), None]),
+    ("lift_gemv batch 17", "lq_lift_gemv", [_c(P), 0, 17, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 8, 1536,
+                                            _c(P), _c(P), None]),
+    ("lift_gemv K mismatch", "lq_lift_gemv", [_c(P), 0, 1, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 8, 1504,
+                                              _c(P), _c(P), None]),
+    ("lift_gemv null o", "lq_lift_gemv", [_c(P), 0, 1, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 8, 1536,
+                                          _c(P), None, None]),
+    ("lift_gemv misaligned u", "lq_lift_gemv", [_c(P), 0, 1, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 8, 1536,
+                                                _c(MIS), _c(P), None]),
+    ("lift_gemv out 0", "lq_lift_gemv", [_c(P), 0, 1, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 0, 1536,
+                                         _c(P), _c(P), None]),
     ("gemm tokens 0", "lq_gemm", [_c(P), _c(P), 8, 64, _c(P), 0, _c(P), None]),
     ("gemm K<32", "lq_gemm", [_c(P), _c(P), 8, 0, _c(P), 4, _c(P), None]),
     ("gemm null o", "lq_gemm", [_c(P), _c(P), 8, 64, _c(P), 4, None, None]),

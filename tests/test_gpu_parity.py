@@ -224,6 +224,42 @@ def test_sweep_decode_sampled_rows(lq, D):
     assert rel_err(o[:, rows], want) <= 1e-5
 
 
+# ------------------------------------------------------------------ one-call decode step
+
+def _fused(lq, L):
+    t = None if L.tinv is None else dev(L.tinv)
+    return lq.lift_gemv(dev(L.a), dev(L.M), dev(L.packed), dev(L.s), L.cfg.K, tinv=t)
+
+
+@pytest.mark.parametrize("name,batch", [("tiny", 1), ("tiny", 2), ("tiny", 3), ("decode_lq24_10", 1),
+                                        ("decode_lq24_10", 2), ("decode_lq20_8", 1), ("sweep_lq19_8", 1),
+                                        ("decode_lq20_8", 4)])
+def test_fused_step_equals_two_calls(lq, name, batch):
+    """lq_lift_gemv gives exactly the results of lq_lift_activations followed by lq_gemv."""
+    L = make_layer(CONFIGS[name], batch)
+    u_f, o_f = _fused(lq, L)
+    u = _gpu_u(lq, L)
+    o = lq.gemv(dev(L.packed), dev(L.s), u)
+    assert np.array_equal(host(u_f), host(u))
+    assert np.array_equal(host(o_f), host(o))
+
+
+def test_fused_step_vs_oracle_alternating_layers(lq):
+    """One-call decode step against the oracle, alternating a small and a large
+    layer (32 and 148 CTAs)."""
+    small = make_layer(CONFIGS["tiny"], 2)
+    big = make_layer(CONFIGS["decode_lq24_10"], 1)
+    _, want_small = oracle.forward(small.packed, small.s, oracle.to_f64(small.a), None, oracle.to_f64(small.M),
+                                   small.cfg.K)
+    rows = _sample_rows(big.cfg.out, 512, 5)
+    want_big = oracle.contract_rows(big.packed, big.s, _oracle_u(big), rows)
+    for _ in range(3):
+        _, o = _fused(lq, small)
+        assert rel_err(host(o), want_small) <= 1e-5
+        _, o = _fused(lq, big)
+        assert rel_err(host(o)[:, rows], want_big) <= 1e-5
+
+
 # ------------------------------------------------------------------ prefill GEMM
 
 @pytest.mark.parametrize("out,K,tokens", [(300, 1536, 300), (128, 64, 256), (129, 1568, 7), (1, 32, 1),
