@@ -20,6 +20,8 @@
 // Accumulation is fp32; bf16 output rounds to nearest even.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "lq_internal.h"
 #include "lq_lift_common.cuh"
 
@@ -299,11 +301,193 @@ __global__ void __launch_bounds__(256) lift_prefill_kernel(LiftArgs p) {
     lift_and_store<PRE_TB, PRE_TT>(p, r, Ms, aps, t0, nt);
 }
 
+// ------------------------------------------------ prefill variant, register tiled
+// For whitening blocks of 16..128 channels (tblk % 8 == 0): a CTA owns G
+// consecutive d-blocks (C <= min(120, tblk) channels, so they touch at most two
+// whitening blocks) and 64 tokens. T^-1 rows and the activations of both
+// whitening blocks are staged transposed in shared memory; each thread forms
+// a' for 4 channels x 8 tokens (32 accumulators, three 16-byte shared loads per
+// 32 FMAs), then the lift reads a' from shared memory. A channel group of 4
+// never straddles whitening blocks: each block's channels are padded to a
+// multiple of 4.
+constexpr int P2_TT = 64;              // tokens per CTA
+constexpr int P2_AP = P2_TT + 4;       // pitch (floats) of a row of staged activations
+constexpr int P2_TP = 132;             // pitch (floats) of a staged T^-1 column (<= 128 padded channels)
+constexpr int P2_CMAX = 120;           // channels per CTA
+
+__host__ __device__ inline size_t prefill2_smem(int tblk, int d, int D) {
+    return sizeof(float) * ((size_t)2 * tblk * P2_AP + (size_t)tblk * P2_TP + (((size_t)d * D + 3) & ~(size_t)3));
+}
+
+__global__ void __launch_bounds__(256) lift_prefill2_kernel(LiftArgs p) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // see lift_decode_kernel
+    extern __shared__ __align__(16) float smem[];
+    const int nblocks = p.in / p.d;
+    const int b0 = blockIdx.x * p.G, b1 = min(nblocks, b0 + p.G);
+    const int c0 = b0 * p.d, C = (b1 - b0) * p.d;
+    const int t0 = blockIdx.y * P2_TT, nt = min(P2_TT, p.batch - t0);
+    const int kb0 = c0 / p.tblk;                          // first whitening block touched
+    const int split = min(C, (kb0 + 1) * p.tblk - c0);    // channels [0, split) lie in block kb0
+    const int PA = (split + 3) & ~3, PB = (C - split + 3) & ~3;
+    const int nbl = split < C ? 2 : 1;
+    float* as = smem;                                   // [2][tblk][P2_AP]: a[t][block bl, j]
+    float* Ts = as + 2 * p.tblk * P2_AP;               // [tblk][P2_TP]: T^-1[c][j] at [j][padded c]
+    float* Ms = Ts + p.tblk * P2_TP;                   // [d*D]
+    float* aps = as;                                    // [C][P2_AP]: a' (reuses the activation area)
+
+    for (int i = threadIdx.x; i < p.d * p.D; i += blockDim.x) Ms[i] = __ldg(p.M + i);
+    // Activations: chunk = 8 consecutive channels of one token (one 16-byte load
+    // of bf16, two of fp32); lanes run over tokens, so the transposed stores
+    // are conflict-free. Eight chunks per thread are requested before any store.
+    {
+        const int jgs = p.tblk >> 3;                     // chunks per whitening block and token
+        const int nchunk = nbl * jgs * P2_TT;
+        for (int base = threadIdx.x; base < nchunk; base += 8 * 256) {
+            float v[8][8];
+#pragma unroll
+            for (int u8 = 0; u8 < 8; ++u8) {
+                const int i = base + u8 * 256, t = i % P2_TT, r = i / P2_TT;
+                const int jg = r % jgs, bl2 = r / jgs;
+                const long long idx = (long long)(t0 + t) * p.in + (kb0 + bl2) * p.tblk + 8 * jg;
+                if (i < nchunk && t < nt) {
+                    if (p.a_bf16) {
+                        const uint4 h = __ldg(reinterpret_cast<const uint4*>(
+                            reinterpret_cast<const unsigned short*>(p.a) + idx));
+                        const uint32_t w[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            v[u8][2 * q] = __uint_as_float(w[q] << 16);
+                            v[u8][2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
+                        }
+                    } else {
+                        const float4 f0 = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.a) + idx));
+                        const float4 f1 =
+                            __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.a) + idx) + 1);
+                        v[u8][0] = f0.x; v[u8][1] = f0.y; v[u8][2] = f0.z; v[u8][3] = f0.w;
+                        v[u8][4] = f1.x; v[u8][5] = f1.y; v[u8][6] = f1.z; v[u8][7] = f1.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) v[u8][q] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int u8 = 0; u8 < 8; ++u8) {
+                const int i = base + u8 * 256, t = i % P2_TT, r = i / P2_TT;
+                const int jg = r % jgs, bl2 = r / jgs;
+                if (i < nchunk) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) as[(bl2 * p.tblk + 8 * jg + q) * P2_AP + t] = v[u8][q];
+                }
+            }
+        }
+    }
+    // T^-1 rows: chunk = 4 consecutive j of one padded channel (one 16-byte
+    // load); lanes run over channels, so the transposed stores are conflict-free.
+    {
+        const int j4s = p.tblk >> 2;
+        const int nchunk = 128 * j4s;                    // padded channels 0..127 (those >= PA + PB are zero)
+        for (int base = threadIdx.x; base < nchunk; base += 8 * 256) {
+            float4 v[8];
+#pragma unroll
+            for (int u8 = 0; u8 < 8; ++u8) {
+                const int i = base + u8 * 256, pc = i & 127, j4 = i >> 7;
+                const int lc = pc < PA ? pc : split + (pc - PA);
+                const bool valid = i < nchunk && (pc < PA ? pc < split : pc < PA + PB && lc < C);
+                v[u8] = valid ? __ldg(reinterpret_cast<const float4*>(p.tinv + (long long)(c0 + lc) * p.tblk) + j4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u8 = 0; u8 < 8; ++u8) {
+                const int i = base + u8 * 256, pc = i & 127, j4 = i >> 7;
+                if (i < nchunk) {
+                    float* dst = Ts + 4 * j4 * P2_TP + pc;
+                    dst[0] = v[u8].x;
+                    dst[P2_TP] = v[u8].y;
+                    dst[2 * P2_TP] = v[u8].z;
+                    dst[3 * P2_TP] = v[u8].w;
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // a' for 4 padded channels x 8 tokens per thread; a warp holds 4 channel
+    // groups x 8 token groups (broadcast-friendly shared loads)
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int cg = warp * 4 + (lane >> 3), tg = lane & 7;
+    const int pc0 = 4 * cg;
+    const bool active = pc0 < PA + PB;
+    const int bl = pc0 < PA ? 0 : 1;
+    float acc[4][8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int t = 0; t < 8; ++t) acc[q][t] = 0.f;
+    if (active) {
+        const float* ab = as + bl * p.tblk * P2_AP + 8 * tg;
+        const float* tb = Ts + pc0;
+#pragma unroll 4
+        for (int j = 0; j < p.tblk; ++j) {
+            const float4 x0 = *reinterpret_cast<const float4*>(ab + j * P2_AP);
+            const float4 x1 = *reinterpret_cast<const float4*>(ab + j * P2_AP + 4);
+            const float4 w = *reinterpret_cast<const float4*>(tb + j * P2_TP);
+            const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            const float ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int t = 0; t < 8; ++t) acc[q][t] = fmaf(ws[q], xs[t], acc[q][t]);
+        }
+    }
+    __syncthreads();  // the activation area becomes a'
+    if (active) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int pc = pc0 + q;
+            const int lc = pc < PA ? pc : split + (pc - PA);
+            if ((pc < PA ? pc < split : lc < C)) {
+                float* dst = aps + lc * P2_AP + 8 * tg;
+                *reinterpret_cast<float4*>(dst) = make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
+                *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[q][4], acc[q][5], acc[q][6], acc[q][7]);
+            }
+        }
+    }
+    __syncthreads();
+
+    // lift: item = (lifted coordinate k of this CTA, token group of 8)
+    const int nk = (b1 - b0) * p.D;
+    for (int item = threadIdx.x; item < nk * (P2_TT / 8); item += blockDim.x) {
+        const int kl = item % nk, g8 = item / nk;
+        const int bl2 = kl / p.D, jj = kl - bl2 * p.D;
+        float o[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) o[t] = 0.f;
+        for (int i = 0; i < p.d; ++i) {
+            const float m = Ms[i * p.D + jj];
+            const float* ar = aps + (bl2 * p.d + i) * P2_AP + 8 * g8;
+            const float4 x0 = *reinterpret_cast<const float4*>(ar);
+            const float4 x1 = *reinterpret_cast<const float4*>(ar + 4);
+            o[0] = fmaf(m, x0.x, o[0]); o[1] = fmaf(m, x0.y, o[1]); o[2] = fmaf(m, x0.z, o[2]); o[3] = fmaf(m, x0.w, o[3]);
+            o[4] = fmaf(m, x1.x, o[4]); o[5] = fmaf(m, x1.y, o[5]); o[6] = fmaf(m, x1.z, o[6]); o[7] = fmaf(m, x1.w, o[7]);
+        }
+        const long long kk = (long long)b0 * p.D + kl;
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+            if (8 * g8 + t < nt) store_u(p.u, p.u_bf16, (long long)(t0 + 8 * g8 + t) * p.K + kk, o[t]);
+    }
+    if (blockIdx.x == gridDim.x - 1) {  // zero the padded tail of the lifted axis
+        const int kreal = nblocks * p.D, npad = p.K - kreal;
+        for (int i = threadIdx.x; i < npad * nt; i += blockDim.x)
+            store_u(p.u, p.u_bf16, (long long)(t0 + i / npad) * p.K + kreal + i % npad, 0.f);
+    }
+}
+
 // Raise a kernel's dynamic shared-memory limit once per device to the largest
 // size requested so far (cudaFuncSetAttribute is not a stream operation, so
 // repeated calls are avoided on launch paths that may be graph-captured).
 cudaError_t raise_smem_limit(const void* fn, size_t bytes, int which) {
-    static size_t granted[2][64] = {};
+    static size_t granted[3][64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && granted[which][dev] >= bytes) return cudaSuccess;
@@ -364,6 +548,15 @@ cudaError_t launch_lift(const void* a, bool a_bf16, int batch, int in, const flo
             if (e != cudaSuccess) return e;
         }
         lift_decode_kernel<<<grid, 256, smem, st>>>(p);
+    } else if (tinv && tblk % 8 == 0 && tblk >= 16 && tblk <= 128 && d <= P2_CMAX && d <= tblk &&
+               prefill2_smem(tblk, d, D) <= 227 * 1024) {
+        LiftArgs q = p;
+        q.G = std::max(1, std::min(P2_CMAX, tblk) / d);
+        const dim3 g2((nblocks + q.G - 1) / q.G, (batch + P2_TT - 1) / P2_TT);
+        const size_t sm2 = prefill2_smem(tblk, d, D);
+        cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(lift_prefill2_kernel), sm2, 2);
+        if (e != cudaSuccess) return e;
+        lift_prefill2_kernel<<<g2, 256, sm2, st>>>(q);
     } else {
         grid.y = (batch + PRE_TB - 1) / PRE_TB;
         smem = sizeof(float) * (mpad + (size_t)span * PRE_TB + (size_t)C * PRE_TB +

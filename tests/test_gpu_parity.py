@@ -118,6 +118,10 @@ def test_lift_padding_and_small_blocks(lq):
     (600, 5, 9, 20, 2, True, "bf16"),      # bf16 lifted output from the decode path
     (512, 16, 64, 0, 4, False, "f32"),     # T = identity
     (1280, 20, 40, 128, 2, True, "f32"),   # d > 16: the shared-memory decode kernel
+    (960, 10, 24, 96, 70, True, "bf16"),   # prefill tiles: blocks straddling 96-wide whitening blocks, ragged tokens
+    (1024, 8, 20, 64, 130, False, "bf16"), # prefill tiles, 64-wide whitening blocks
+    (1024, 8, 20, 128, 33, True, "f32"),   # prefill tiles with fp32 output
+    (768, 6, 14, 256, 40, True, "bf16"),   # 256-wide whitening blocks: the shared-memory prefill kernel
 ])
 def test_lift_decode_shapes(lq, in_dim, d, D, tblk, batch, a_bf16, u_dtype):
     from datagen.inputs import bf16_bits_from_f32
