@@ -311,12 +311,19 @@ __global__ void __launch_bounds__(256) lift_prefill_kernel(LiftArgs p) {
 // never straddles whitening blocks: each block's channels are padded to a
 // multiple of 4.
 constexpr int P2_TT = 64;              // tokens per CTA
-constexpr int P2_AP = P2_TT + 4;       // pitch (floats) of a row of staged activations
+constexpr int P2_AP = 76;              // pitch (floats) of a row of 64 staged tokens (see p2_pos)
 constexpr int P2_TP = 132;             // pitch (floats) of a staged T^-1 column (<= 128 padded channels)
 constexpr int P2_CMAX = 120;           // channels per CTA
+constexpr int P2_JC = 64;              // whitening-block columns staged at a time
+
+// Position of token t in a staged row: token group g = t/8 keeps its first four
+// tokens at 4g and its last four at 36 + 4g, so the eight 16-byte chunks that
+// the eight token groups of a quarter-warp read fall in distinct bank groups.
+__device__ __forceinline__ int p2_pos(int t) { return ((t >> 2) & 1) * 36 + (t >> 3) * 4 + (t & 3); }
 
 __host__ __device__ inline size_t prefill2_smem(int tblk, int d, int D) {
-    return sizeof(float) * ((size_t)2 * tblk * P2_AP + (size_t)tblk * P2_TP + (((size_t)d * D + 3) & ~(size_t)3));
+    const size_t jc = tblk < P2_JC ? tblk : P2_JC;
+    return sizeof(float) * ((size_t)2 * jc * P2_AP + (size_t)jc * P2_TP + (((size_t)d * D + 3) & ~(size_t)3));
 }
 
 __global__ void __launch_bounds__(256) lift_prefill2_kernel(LiftArgs p) {
@@ -330,88 +337,13 @@ __global__ void __launch_bounds__(256) lift_prefill2_kernel(LiftArgs p) {
     const int split = min(C, (kb0 + 1) * p.tblk - c0);    // channels [0, split) lie in block kb0
     const int PA = (split + 3) & ~3, PB = (C - split + 3) & ~3;
     const int nbl = split < C ? 2 : 1;
-    float* as = smem;                                   // [2][tblk][P2_AP]: a[t][block bl, j]
-    float* Ts = as + 2 * p.tblk * P2_AP;               // [tblk][P2_TP]: T^-1[c][j] at [j][padded c]
-    float* Ms = Ts + p.tblk * P2_TP;                   // [d*D]
+    const int JC = min(P2_JC, p.tblk);                 // columns j staged per pass
+    float* as = smem;                                   // [2][JC][P2_AP]: a[t][block bl, j0 + j]
+    float* Ts = as + 2 * JC * P2_AP;                   // [JC][P2_TP]: T^-1[c][j0 + j] at [j][padded c]
+    float* Ms = Ts + JC * P2_TP;                       // [d*D]
     float* aps = as;                                    // [C][P2_AP]: a' (reuses the activation area)
 
     for (int i = threadIdx.x; i < p.d * p.D; i += blockDim.x) Ms[i] = __ldg(p.M + i);
-    // Activations: chunk = 8 consecutive channels of one token (one 16-byte load
-    // of bf16, two of fp32); lanes run over tokens, so the transposed stores
-    // are conflict-free. Eight chunks per thread are requested before any store.
-    {
-        const int jgs = p.tblk >> 3;                     // chunks per whitening block and token
-        const int nchunk = nbl * jgs * P2_TT;
-        for (int base = threadIdx.x; base < nchunk; base += 8 * 256) {
-            float v[8][8];
-#pragma unroll
-            for (int u8 = 0; u8 < 8; ++u8) {
-                const int i = base + u8 * 256, t = i % P2_TT, r = i / P2_TT;
-                const int jg = r % jgs, bl2 = r / jgs;
-                const long long idx = (long long)(t0 + t) * p.in + (kb0 + bl2) * p.tblk + 8 * jg;
-                if (i < nchunk && t < nt) {
-                    if (p.a_bf16) {
-                        const uint4 h = __ldg(reinterpret_cast<const uint4*>(
-                            reinterpret_cast<const unsigned short*>(p.a) + idx));
-                        const uint32_t w[4] = {h.x, h.y, h.z, h.w};
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            v[u8][2 * q] = __uint_as_float(w[q] << 16);
-                            v[u8][2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
-                        }
-                    } else {
-                        const float4 f0 = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.a) + idx));
-                        const float4 f1 =
-                            __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.a) + idx) + 1);
-                        v[u8][0] = f0.x; v[u8][1] = f0.y; v[u8][2] = f0.z; v[u8][3] = f0.w;
-                        v[u8][4] = f1.x; v[u8][5] = f1.y; v[u8][6] = f1.z; v[u8][7] = f1.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) v[u8][q] = 0.f;
-                }
-            }
-#pragma unroll
-            for (int u8 = 0; u8 < 8; ++u8) {
-                const int i = base + u8 * 256, t = i % P2_TT, r = i / P2_TT;
-                const int jg = r % jgs, bl2 = r / jgs;
-                if (i < nchunk) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) as[(bl2 * p.tblk + 8 * jg + q) * P2_AP + t] = v[u8][q];
-                }
-            }
-        }
-    }
-    // T^-1 rows: chunk = 4 consecutive j of one padded channel (one 16-byte
-    // load); lanes run over channels, so the transposed stores are conflict-free.
-    {
-        const int j4s = p.tblk >> 2;
-        const int nchunk = 128 * j4s;                    // padded channels 0..127 (those >= PA + PB are zero)
-        for (int base = threadIdx.x; base < nchunk; base += 8 * 256) {
-            float4 v[8];
-#pragma unroll
-            for (int u8 = 0; u8 < 8; ++u8) {
-                const int i = base + u8 * 256, pc = i & 127, j4 = i >> 7;
-                const int lc = pc < PA ? pc : split + (pc - PA);
-                const bool valid = i < nchunk && (pc < PA ? pc < split : pc < PA + PB && lc < C);
-                v[u8] = valid ? __ldg(reinterpret_cast<const float4*>(p.tinv + (long long)(c0 + lc) * p.tblk) + j4)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u8 = 0; u8 < 8; ++u8) {
-                const int i = base + u8 * 256, pc = i & 127, j4 = i >> 7;
-                if (i < nchunk) {
-                    float* dst = Ts + 4 * j4 * P2_TP + pc;
-                    dst[0] = v[u8].x;
-                    dst[P2_TP] = v[u8].y;
-                    dst[2 * P2_TP] = v[u8].z;
-                    dst[3 * P2_TP] = v[u8].w;
-                }
-            }
-        }
-    }
-    __syncthreads();
-
     // a' for 4 padded channels x 8 tokens per thread; a warp holds 4 channel
     // groups x 8 token groups (broadcast-friendly shared loads)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -424,20 +356,99 @@ __global__ void __launch_bounds__(256) lift_prefill2_kernel(LiftArgs p) {
     for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int t = 0; t < 8; ++t) acc[q][t] = 0.f;
-    if (active) {
-        const float* ab = as + bl * p.tblk * P2_AP + 8 * tg;
-        const float* tb = Ts + pc0;
+    for (int j0 = 0; j0 < p.tblk; j0 += JC) {
+        const int jc = min(JC, p.tblk - j0);  // a multiple of 8
+        if (j0) __syncthreads();  // the previous columns have been consumed
+        // Activations: chunk = 8 consecutive channels of one token (one 16-byte load
+        // of bf16, two of fp32); lanes run over tokens, so the transposed stores
+        // are conflict-free. Eight chunks per thread are requested before any store.
+        {
+            const int jgs = jc >> 3;                         // chunks per whitening block and token
+            const int nchunk = nbl * jgs * P2_TT;
+            for (int base = threadIdx.x; base < nchunk; base += 8 * 256) {
+                float v[8][8];
+#pragma unroll
+                for (int u8 = 0; u8 < 8; ++u8) {
+                    const int i = base + u8 * 256, t = i % P2_TT, r = i / P2_TT;
+                    const int jg = r % jgs, bl2 = r / jgs;
+                    const long long idx = (long long)(t0 + t) * p.in + (kb0 + bl2) * p.tblk + j0 + 8 * jg;
+                    if (i < nchunk && t < nt) {
+                        if (p.a_bf16) {
+                            const uint4 h = __ldg(reinterpret_cast<const uint4*>(
+                                reinterpret_cast<const unsigned short*>(p.a) + idx));
+                            const uint32_t w[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                v[u8][2 * q] = __uint_as_float(w[q] << 16);
+                                v[u8][2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
+                            }
+                        } else {
+                            const float4 f0 = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.a) + idx));
+                            const float4 f1 =
+                                __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.a) + idx) + 1);
+                            v[u8][0] = f0.x; v[u8][1] = f0.y; v[u8][2] = f0.z; v[u8][3] = f0.w;
+                            v[u8][4] = f1.x; v[u8][5] = f1.y; v[u8][6] = f1.z; v[u8][7] = f1.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) v[u8][q] = 0.f;
+                    }
+                }
+#pragma unroll
+                for (int u8 = 0; u8 < 8; ++u8) {
+                    const int i = base + u8 * 256, t = i % P2_TT, r = i / P2_TT;
+                    const int jg = r % jgs, bl2 = r / jgs;
+                    if (i < nchunk) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) as[(bl2 * JC + 8 * jg + q) * P2_AP + p2_pos(t)] = v[u8][q];
+                    }
+                }
+            }
+        }
+        // T^-1 rows: chunk = 4 consecutive j of one padded channel (one 16-byte
+        // load); lanes run over channels, so the transposed stores are conflict-free.
+        {
+            const int j4s = jc >> 2;
+            const int nchunk = 128 * j4s;                    // padded channels 0..127 (those >= PA + PB are zero)
+            for (int base = threadIdx.x; base < nchunk; base += 8 * 256) {
+                float4 v[8];
+#pragma unroll
+                for (int u8 = 0; u8 < 8; ++u8) {
+                    const int i = base + u8 * 256, pc = i & 127, j4 = i >> 7;
+                    const int lc = pc < PA ? pc : split + (pc - PA);
+                    const bool valid = i < nchunk && (pc < PA ? pc < split : pc < PA + PB && lc < C);
+                    v[u8] = valid ? __ldg(reinterpret_cast<const float4*>(p.tinv + (long long)(c0 + lc) * p.tblk + j0) + j4)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u8 = 0; u8 < 8; ++u8) {
+                    const int i = base + u8 * 256, pc = i & 127, j4 = i >> 7;
+                    if (i < nchunk) {
+                        float* dst = Ts + 4 * j4 * P2_TP + pc;
+                        dst[0] = v[u8].x;
+                        dst[P2_TP] = v[u8].y;
+                        dst[2 * P2_TP] = v[u8].z;
+                        dst[3 * P2_TP] = v[u8].w;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (active) {
+            const float* ab = as + bl * JC * P2_AP + 4 * tg;
+            const float* tb = Ts + pc0;
 #pragma unroll 4
-        for (int j = 0; j < p.tblk; ++j) {
-            const float4 x0 = *reinterpret_cast<const float4*>(ab + j * P2_AP);
-            const float4 x1 = *reinterpret_cast<const float4*>(ab + j * P2_AP + 4);
-            const float4 w = *reinterpret_cast<const float4*>(tb + j * P2_TP);
-            const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-            const float ws[4] = {w.x, w.y, w.z, w.w};
+            for (int j = 0; j < jc; ++j) {
+                const float4 x0 = *reinterpret_cast<const float4*>(ab + j * P2_AP);
+                const float4 x1 = *reinterpret_cast<const float4*>(ab + j * P2_AP + 36);
+                const float4 w = *reinterpret_cast<const float4*>(tb + j * P2_TP);
+                const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                const float ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+                for (int q = 0; q < 4; ++q)
 #pragma unroll
-                for (int t = 0; t < 8; ++t) acc[q][t] = fmaf(ws[q], xs[t], acc[q][t]);
+                    for (int t = 0; t < 8; ++t) acc[q][t] = fmaf(ws[q], xs[t], acc[q][t]);
+            }
         }
     }
     __syncthreads();  // the activation area becomes a'
@@ -447,9 +458,9 @@ __global__ void __launch_bounds__(256) lift_prefill2_kernel(LiftArgs p) {
             const int pc = pc0 + q;
             const int lc = pc < PA ? pc : split + (pc - PA);
             if ((pc < PA ? pc < split : lc < C)) {
-                float* dst = aps + lc * P2_AP + 8 * tg;
+                float* dst = aps + lc * P2_AP + 4 * tg;
                 *reinterpret_cast<float4*>(dst) = make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
-                *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[q][4], acc[q][5], acc[q][6], acc[q][7]);
+                *reinterpret_cast<float4*>(dst + 36) = make_float4(acc[q][4], acc[q][5], acc[q][6], acc[q][7]);
             }
         }
     }
@@ -465,9 +476,9 @@ __global__ void __launch_bounds__(256) lift_prefill2_kernel(LiftArgs p) {
         for (int t = 0; t < 8; ++t) o[t] = 0.f;
         for (int i = 0; i < p.d; ++i) {
             const float m = Ms[i * p.D + jj];
-            const float* ar = aps + (bl2 * p.d + i) * P2_AP + 8 * g8;
+            const float* ar = aps + (bl2 * p.d + i) * P2_AP + 4 * g8;
             const float4 x0 = *reinterpret_cast<const float4*>(ar);
-            const float4 x1 = *reinterpret_cast<const float4*>(ar + 4);
+            const float4 x1 = *reinterpret_cast<const float4*>(ar + 36);
             o[0] = fmaf(m, x0.x, o[0]); o[1] = fmaf(m, x0.y, o[1]); o[2] = fmaf(m, x0.z, o[2]); o[3] = fmaf(m, x0.w, o[3]);
             o[4] = fmaf(m, x1.x, o[4]); o[5] = fmaf(m, x1.y, o[5]); o[6] = fmaf(m, x1.z, o[6]); o[7] = fmaf(m, x1.w, o[7]);
         }
