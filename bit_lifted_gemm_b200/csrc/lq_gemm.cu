@@ -9,9 +9,14 @@
 // is exact; the only rounding is fp32 accumulation (plus the bf16 rounding of
 // u done by the lift).
 //
-// One CTA computes a 128 (rows of W_q) x 256 (tokens) tile, K in steps of 64:
-//   warp 0      TMA producer: u tile [256 tokens][64 k] bf16, 128-byte swizzle
-//   warp 1      TMEM allocator and single-thread UMMA issuer (M=128, N=256, K=16)
+// One CTA computes a 128 (rows of W_q) x BN (tokens) tile, K in steps of 64;
+// BN = 256, or 64 for short token runs (a quarter of the MMA, TMEM and u
+// traffic per k-step). When the tiles cannot fill the SMs, K is split in two:
+// each half scales its partial by s[r] and adds it atomically into o, zeroed
+// first; with exactly two terms the sum does not depend on their order, so
+// the result is deterministic.
+//   warp 0      TMA producer: u tile [BN tokens][64 k] bf16, 128-byte swizzle
+//   warp 1      TMEM allocator and single-thread UMMA issuer (M=128, N=BN, K=16)
 //   warps 2..5  one thread per tile row: load that row's two sign words for the
 //               k-step, expand the 64 bits to +-1 bf16 in registers and store
 //               them in the same 128-byte-swizzled K-major layout the TMA uses;
@@ -29,13 +34,16 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BK = 64, STAGES = 4;
 constexpr int A_STAGE = BM * BK * 2;   // 16 KB
-constexpr int B_STAGE = BN * BK * 2;   // 32 KB
-constexpr int TMEM_COLS = 256;         // fp32 accumulator, 128 lanes x 256 columns
 constexpr int THREADS = 192;
 constexpr int UNPACK_THREADS = 128;
-constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * (A_STAGE + B_STAGE) + 256;
+template <int BN>
+struct Tile {
+    static constexpr int B_STAGE = BN * BK * 2;  // 32 KB (BN 256) or 8 KB (BN 64)
+    static constexpr int TMEM_COLS = BN;         // fp32 accumulator, 128 lanes x BN columns
+    static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * (A_STAGE + B_STAGE) + 256;
+};
 
 // Expand 16 sign bits (bit i = element i of a k-run) into 8 bf16x2 words:
 // word i holds elements (2i, 2i+1) as +1.0 (0x3F80) or -1.0 (0xBF80).
@@ -52,10 +60,12 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
+template <int BN>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_u, const uint32_t* __restrict__ packed,
                 const float* __restrict__ s, int out, int K, int tokens, float* __restrict__ o,
                 unsigned* status) {
+    constexpr int B_STAGE = Tile<BN>::B_STAGE, TMEM_COLS = Tile<BN>::TMEM_COLS;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned for the 128-byte swizzle; offsetting the array itself
     // keeps derived pointers in the shared address space
@@ -69,7 +79,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
-    const int nkb = (K + BK - 1) / BK;
+    // K split in gridDim.z (1 or 2) parts: this CTA takes k-blocks [kb_lo, kb_hi),
+    // the split on a multiple of 8 k-blocks (aligned 16-word groups of sign words)
+    const int nkb_all = (K + BK - 1) / BK;
+    const int kb_lo = blockIdx.z == 0 ? 0 : (int)((long long)blockIdx.z * nkb_all / gridDim.z) & ~7;
+    const int kb_hi = blockIdx.z + 1 == gridDim.z ? nkb_all : (int)((long long)(blockIdx.z + 1) * nkb_all / gridDim.z) & ~7;
+    const int nkb = kb_hi - kb_lo;
+    const bool split = gridDim.z > 1;
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
@@ -100,7 +116,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     break;
                 }
                 mbar_arrive_expect_tx(full0 + 8 * st, B_STAGE);
-                tma_load_2d(smem_addr(sB + st * B_STAGE), &tmap_u, kb * BK, n0, full0 + 8 * st);
+                tma_load_2d(smem_addr(sB + st * B_STAGE), &tmap_u, (kb_lo + kb) * BK, n0, full0 + 8 * st);
                 issued = kb + 1;
             }
             // Do not leave copies in flight: wait (bounded) for the last load of each stage.
@@ -134,25 +150,55 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t* prow = packed + (long long)grow * kw;
         const uint32_t sw = row & 7;
         const uint32_t row_off = (row >> 3) * 1024 + (row & 7) * 128;
-        for (int kb = 0; kb < nkb; ++kb) {
-            const int st = kb % STAGES, round = kb / STAGES;
-            const uint32_t w0 = 2 * kb < kw ? __ldg(prow + 2 * kb) : 0u;
-            const uint32_t w1 = 2 * kb + 1 < kw ? __ldg(prow + 2 * kb + 1) : 0u;  // u is zero past K
-            uint32_t v[32];
-            expand16(w0 & 0xFFFFu, v);
-            expand16(w0 >> 16, v + 8);
-            expand16(w1 & 0xFFFFu, v + 16);
-            expand16(w1 >> 16, v + 24);
-            if (round > 0 && !mbar_wait(empty0 + 8 * st, (round - 1) & 1, status)) {
-                *abort_flag = 1;
-                break;
-            }
-            const uint32_t dst = smem_addr(sA + st * A_STAGE) + row_off;
+        // The row's sign words arrive 8 k-steps (16 words) at a time, the next
+        // group requested before the current one is expanded, so the unpackers
+        // do not wait a memory round trip per k-step.
+        const bool vec = (kw & 3) == 0;  // 16-byte aligned rows
+        auto load16 = [&](int kg0, uint32_t (&w)[16]) {
+            if (vec && (kg0 & 1) == 0 && 2 * kg0 + 16 <= kw) {
+                const uint4* src = reinterpret_cast<const uint4*>(prow + 2 * kg0);
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                st_shared_v4(dst + ((c ^ sw) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-            fence_proxy_async_smem();
-            mbar_arrive(full0 + 8 * st);
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 x = __ldg(src + q);
+                    w[4 * q] = x.x;
+                    w[4 * q + 1] = x.y;
+                    w[4 * q + 2] = x.z;
+                    w[4 * q + 3] = x.w;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) w[q] = 2 * kg0 + q < kw ? __ldg(prow + 2 * kg0 + q) : 0u;  // u is zero past K
+            }
+        };
+        uint32_t cur[16], nxt[16];
+        load16(kb_lo, cur);
+        bool stop = false;
+        for (int kb0 = 0; kb0 < nkb && !stop; kb0 += 8) {
+            if (kb0 + 8 < nkb) load16(kb_lo + kb0 + 8, nxt);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int kb = kb0 + kk;
+                if (kb >= nkb || stop) break;
+                const int st = kb % STAGES, round = kb / STAGES;
+                uint32_t v[32];
+                expand16(cur[2 * kk] & 0xFFFFu, v);
+                expand16(cur[2 * kk] >> 16, v + 8);
+                expand16(cur[2 * kk + 1] & 0xFFFFu, v + 16);
+                expand16(cur[2 * kk + 1] >> 16, v + 24);
+                if (round > 0 && !mbar_wait(empty0 + 8 * st, (round - 1) & 1, status)) {
+                    *abort_flag = 1;
+                    stop = true;
+                    break;
+                }
+                const uint32_t dst = smem_addr(sA + st * A_STAGE) + row_off;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_shared_v4(dst + ((c ^ sw) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                fence_proxy_async_smem();
+                mbar_arrive(full0 + 8 * st);
+            }
+#pragma unroll
+            for (int q = 0; q < 16; ++q) cur[q] = nxt[q];
         }
 
         // ---- epilogue: TMEM -> registers -> s[r] * acc -> o[t][r]
@@ -172,7 +218,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int n = n0 + c0 + j;
-                        if (n < tokens) o[(long long)n * out + m] = sr * __uint_as_float(v[j]);
+                        if (n < tokens) {
+                            if (split)
+                                atomicAdd(o + (long long)n * out + m, sr * __uint_as_float(v[j]));
+                            else
+                                o[(long long)n * out + m] = sr * __uint_as_float(v[j]);
+                        }
                     }
                 }
             }
@@ -203,10 +254,9 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-}  // namespace
-
-cudaError_t launch_gemm(const uint32_t* packed, const float* s, int out, int K, const uint16_t* u_bf16,
-                        int tokens, float* o, unsigned* status, cudaStream_t st) {
+template <int BN>
+cudaError_t launch_tile(const uint32_t* packed, const float* s, int out, int K, const uint16_t* u_bf16, int tokens,
+                        float* o, unsigned* status, cudaStream_t st, int num_sms) {
     EncodeTiledFn encode = encode_fn();
     if (!encode) return cudaErrorNotSupported;
     CUtensorMap map;
@@ -218,18 +268,36 @@ cudaError_t launch_gemm(const uint32_t* packed, const float* s, int out, int K, 
                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)Tile<BN>::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    dim3 grid((out + BM - 1) / BM, (tokens + BN - 1) / BN);
-    gemm_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(map, packed, s, out, K, tokens, o, status);
+    dim3 grid((out + BM - 1) / BM, (tokens + BN - 1) / BN, 1);
+    const int nkb = (K + BK - 1) / BK;
+    if ((long long)grid.x * grid.y < num_sms && nkb >= 16) {  // too few tiles for the SMs: split K in two
+        grid.z = 2;
+        cudaError_t e = cudaMemsetAsync(o, 0, (size_t)tokens * out * sizeof(float), st);
+        if (e != cudaSuccess) return e;
+    }
+    gemm_kernel<BN><<<grid, THREADS, Tile<BN>::SMEM_BYTES, st>>>(map, packed, s, out, K, tokens, o, status);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const uint32_t* packed, const float* s, int out, int K, const uint16_t* u_bf16,
+                        int tokens, float* o, unsigned* status, cudaStream_t st) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // short token runs: 64-token tiles (less idle MMA width and u traffic)
+    if (tokens <= 64) return launch_tile<64>(packed, s, out, K, u_bf16, tokens, o, status, st, sms);
+    return launch_tile<256>(packed, s, out, K, u_bf16, tokens, o, status, st, sms);
 }
 
 }  // namespace lq
