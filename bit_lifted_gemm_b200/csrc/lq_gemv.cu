@@ -584,9 +584,10 @@ int max_segments(int grid, int ngroups, int tpg) {
     return (int)((len + tpg - 1) / tpg + 1);
 }
 
-// One CTA per SM (or per group when there are fewer groups); the widest K chunk
-// and up to two columns whose digit planes fit in shared memory, preferring a
-// deep ring, then u staged by TMA.
+// One CTA per SM (or per group when there are fewer groups). Preference: up to
+// two columns per pass, then a deep ring (three tiles in flight per warp), then
+// the widest K chunk whose digit planes fit in shared memory (a second launch
+// costs less than a shallow ring), then u staged by TMA.
 Plan make_plan(int out, int kw, int batch) {
     const int ngroups = (out + 15) / 16;
     const int kwp = (kw + 15) / 16 * 16;
@@ -594,25 +595,27 @@ Plan make_plan(int out, int kw, int batch) {
     pl.tma = (kw % 4) == 0;
     pl.ts = pl.tma && kw % 16 == 0 ? 2 : 1;
     pl.grid = std::min(num_sms(), ngroups);
-    for (int nchunks = 1;; ++nchunks) {
-        pl.kwc = ((kwp + nchunks - 1) / nchunks + 15) / 16 * 16;
-        pl.pitch = plane_pitch(pl.kwc);
-        const int tpg = (pl.kwc / kStepWords + pl.ts - 1) / pl.ts;
-        pl.maxseg = max_segments(pl.grid, ngroups, tpg);
-        for (int cols = std::min(kMaxColsPass, batch); cols >= 1; --cols) {
-            pl.cols = cols;
-            const int nrounds = (cols * pl.kwc + kThreads - 1) / kThreads;
-            for (int deep = pl.tma ? 1 : 0; deep >= 0; --deep) {
-                pl.stages = (pl.ts == 2 ? 2 : 4) * (deep ? 2 : 1);  // the register path is built for 4
+    for (int cols = std::min(kMaxColsPass, batch); cols >= 1; --cols) {
+        pl.cols = cols;
+        for (int deep = pl.tma ? 1 : 0; deep >= 0; --deep) {
+            pl.stages = pl.tma ? (pl.ts == 2 ? 2 : 4) * (deep ? 2 : 1) : 4;  // the register path is built for 4
+            for (int nchunks = 1; nchunks <= (deep ? 2 : 1 << 20); ++nchunks) {
+                pl.kwc = ((kwp + nchunks - 1) / nchunks + 15) / 16 * 16;
+                pl.pitch = plane_pitch(pl.kwc);
+                const int tpg = (pl.kwc / kStepWords + pl.ts - 1) / pl.ts;
+                pl.maxseg = max_segments(pl.grid, ngroups, tpg);
+                const int nrounds = (cols * pl.kwc + kThreads - 1) / kThreads;
                 for (int us = 1; us >= 0; --us) {
                     pl.ustage = us && pl.tma && nrounds <= kMaxRounds;
                     if (us && !pl.ustage) continue;
-                    pl.smem = gemv_layout(pl.ts, pl.stages, pl.tma, pl.ustage, cols, pl.kwc, pl.pitch, pl.maxseg).total;
+                    pl.smem =
+                        gemv_layout(pl.ts, pl.stages, pl.tma, pl.ustage, cols, pl.kwc, pl.pitch, pl.maxseg).total;
                     if (pl.smem <= kSmemBudget) return pl;
                 }
             }
         }
     }
+    return pl;  // not reached: one column with enough chunks always fits
 }
 
 template <int TS, int STAGES, bool TMA, bool USTAGE>
