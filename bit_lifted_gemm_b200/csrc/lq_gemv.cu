@@ -66,6 +66,7 @@ constexpr int kStepWords = 16;    // words per row a warp consumes per step
 constexpr int kStepBytes = 16 * kStepWords * 4;  // one step of 16 rows x 64 bytes
 constexpr int kMaxRounds = 2;     // quantization items per thread kept in registers (staged path)
 constexpr int kUBoxRows = 16;     // words per TMA box of u
+constexpr int kMaxSegSteps = 255;  // steps one 32-bit segment sum holds
 constexpr size_t kSmemBudget = 220 * 1024;
 
 // Digit-plane storage: 16-byte chunks; word pair (x, x+1), x even, occupies the
@@ -484,31 +485,30 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
         }
         if (kfail >= 0) break;
         // ---- segment partial: V = sum_j 2^(7-j) acc_j = 2^7 sum_{bit=1} d per digit
-        // column; gather the three planes of each batch column with shuffles
-        double vreg[4];
+        // column (|V| < 2^23 per step, so 32 bits hold up to 255 steps); gather
+        // the three planes of each batch column with shuffles
+        int vreg[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            long long vv = 0;
+            int vv = acc[0][e];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) vv += (long long)acc[j][e] * (1ll << (7 - j));
-            vreg[e] = (double)vv;
+            for (int j = 1; j < 8; ++j) vv = 2 * vv + acc[j][e];
+            vreg[e] = vv;
         }
         double* dst = part + (size_t)(warp * p.maxseg + seg) * p.ncols * 16;
-        for (int c = 0; c < p.ncols; ++c) {
+#pragma unroll
+        for (int c = 0; c < kMaxColsPass; ++c) {
+            if (c >= p.ncols) break;
 #pragma unroll
             for (int hr = 0; hr < 2; ++hr) {  // rows g (hr = 0) and g + 8
-                double s1 = 0.0;
+                long long s1 = 0;
 #pragma unroll
                 for (int pl = 0; pl < 3; ++pl) {
-                    const int col = 3 * c + pl, e = 2 * hr + (col & 1);
-                    double mine = 0.0;
-#pragma unroll
-                    for (int ee = 0; ee < 4; ++ee)
-                        if (ee == e) mine = vreg[ee];
-                    const double vv = __shfl_sync(0xffffffffu, mine, (lane & ~3) | (col >> 1));
-                    s1 += (pl == 0 ? 1.0 : pl == 1 ? 256.0 : 65536.0) * vv;  // exact: 2^7 sum_{bit=1} u_q
+                    const int col = 3 * c + pl;
+                    const int vv = __shfl_sync(0xffffffffu, vreg[2 * hr + (col & 1)], (lane & ~3) | (col >> 1));
+                    s1 += (long long)vv << (8 * pl);  // exact: 2^7 sum_{bit=1} u_q
                 }
-                if (t == 0) dst[c * 16 + g + 8 * hr] = s1 * (1.0 / 64.0);  // 2 sum_{bit=1} u_q
+                if (t == 0) dst[c * 16 + g + 8 * hr] = (double)s1 * (1.0 / 64.0);  // 2 sum_{bit=1} u_q
             }
         }
     }
@@ -601,6 +601,7 @@ Plan make_plan(int out, int kw, int batch) {
             pl.stages = pl.tma ? (pl.ts == 2 ? 2 : 4) * (deep ? 2 : 1) : 4;  // the register path is built for 4
             for (int nchunks = 1; nchunks <= (deep ? 2 : 1 << 20); ++nchunks) {
                 pl.kwc = ((kwp + nchunks - 1) / nchunks + 15) / 16 * 16;
+                if (pl.kwc > kMaxSegSteps * kStepWords) continue;  // 32-bit segment sums
                 pl.pitch = plane_pitch(pl.kwc);
                 const int tpg = (pl.kwc / kStepWords + pl.ts - 1) / pl.ts;
                 pl.maxseg = max_segments(pl.grid, ngroups, tpg);
