@@ -114,6 +114,11 @@ __device__ __forceinline__ uint4 load_words(const uint32_t* row, int x, int kw) 
     return v;
 }
 
+// floor(i * n / parts) for i <= 256, in 32-bit arithmetic when the product fits.
+__device__ __forceinline__ int split_point(unsigned i, unsigned n, unsigned parts) {
+    return n < (1u << 24) ? (int)(i * n / parts) : (int)((unsigned long long)i * n / parts);
+}
+
 // 2^e as a float for -126 <= e <= 127.
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
 
@@ -283,14 +288,14 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
     uint8_t* smem = smem_raw + ((1024u - (sm100::smem_addr(smem_raw) & 1023u)) & 1023u);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int gbeg = (int)((long long)blockIdx.x * p.ngroups / gridDim.x);
-    const int gend = (int)((long long)(blockIdx.x + 1) * p.ngroups / gridDim.x);
+    const int gbeg = split_point(blockIdx.x, p.ngroups, gridDim.x);
+    const int gend = split_point(blockIdx.x + 1, p.ngroups, gridDim.x);
     const int m0 = 16 * gbeg;
     const int spg = p.kwc / kStepWords;              // steps per group
     const int tpg = (spg + TS - 1) / TS;             // tiles per group
     const int total = (gend - gbeg) * tpg;           // tiles of this CTA
-    const int t0 = (int)((long long)warp * total / kWarps);
-    const int t1 = (int)((long long)(warp + 1) * total / kWarps);
+    const int t0 = split_point(warp, total, kWarps);
+    const int t1 = split_point(warp + 1, total, kWarps);
     const int ndig = 3 * p.ncols;
     constexpr int kTileBytes = TS * kStepBytes;
 
@@ -349,7 +354,7 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
         colmax[threadIdx.x] = 0u;
         sall[threadIdx.x] = 0ull;
     }
-    if (threadIdx.x <= kWarps) wbound[threadIdx.x] = (int)((long long)threadIdx.x * total / kWarps);
+    if (threadIdx.x <= kWarps) wbound[threadIdx.x] = split_point(threadIdx.x, total, kWarps);
     __syncthreads();
 
     // u is written by the kernel before this one on the stream
@@ -478,7 +483,7 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
             }
             mma_step(acc, ca0, cb0, bp);
             bp += binc;
-            if (TS == 2 && xs + 1 < spg) {
+            if (TS == 2) {  // the K chunk of two-step tiles is a multiple of 32 words
                 mma_step(acc, ca1, cb1, bp);
                 bp += binc;
             }
@@ -590,17 +595,18 @@ int max_segments(int grid, int ngroups, int tpg) {
 // costs less than a shallow ring), then u staged by TMA.
 Plan make_plan(int out, int kw, int batch) {
     const int ngroups = (out + 15) / 16;
-    const int kwp = (kw + 15) / 16 * 16;
     Plan pl;
     pl.tma = (kw % 4) == 0;
     pl.ts = pl.tma && kw % 16 == 0 ? 2 : 1;
+    const int q = pl.ts * kStepWords;  // K chunks hold whole tiles (zeros past the row end)
+    const int kwp = (kw + q - 1) / q * q;
     pl.grid = std::min(num_sms(), ngroups);
     for (int cols = std::min(kMaxColsPass, batch); cols >= 1; --cols) {
         pl.cols = cols;
         for (int deep = pl.tma ? 1 : 0; deep >= 0; --deep) {
             pl.stages = pl.tma ? (pl.ts == 2 ? 2 : 4) * (deep ? 2 : 1) : 4;  // the register path is built for 4
             for (int nchunks = 1; nchunks <= (deep ? 2 : 1 << 20); ++nchunks) {
-                pl.kwc = ((kwp + nchunks - 1) / nchunks + 15) / 16 * 16;
+                pl.kwc = ((kwp + nchunks - 1) / nchunks + q - 1) / q * q;
                 if (pl.kwc > kMaxSegSteps * kStepWords) continue;  // 32-bit segment sums
                 pl.pitch = plane_pitch(pl.kwc);
                 const int tpg = (pl.kwc / kStepWords + pl.ts - 1) / pl.ts;
