@@ -98,8 +98,11 @@ int lq_lift_activations(const void* a, int a_dtype, int batch, int in, const flo
     if (batch < 1 || in < 1 || d < 1 || d > 64 || D < 1 || D > 256 || d * D > 4096) return LQ_ERR_INVALID_ARG;
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
     if (tinv && (tblk < 1 || tblk > 256 || in % tblk != 0)) return LQ_ERR_INVALID_ARG;
+    int err = LQ_OK;
+    unsigned* status = status_word(&err);
+    if (!status) return err;
     return from_cuda(lq::launch_lift(a, a_dtype == LQ_BF16, batch, in, tinv, tblk, M, d, D, u, u_dtype == LQ_BF16,
-                                     K, static_cast<cudaStream_t>(stream)));
+                                     K, status, static_cast<cudaStream_t>(stream)));
 }
 
 int lq_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u, int batch, float* o,

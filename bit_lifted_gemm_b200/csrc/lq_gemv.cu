@@ -739,7 +739,7 @@ cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, 
 cudaError_t launch_lift_gemv(const void* a, bool a_bf16, int batch, int in, const float* tinv, int tblk,
                              const float* M, int d, int D, const uint32_t* packed, const float* s, int out, int K,
                              float* u, float* o, unsigned* status, cudaStream_t st) {
-    cudaError_t e = launch_lift(a, a_bf16, batch, in, tinv, tblk, M, d, D, u, false, K, st);
+    cudaError_t e = launch_lift(a, a_bf16, batch, in, tinv, tblk, M, d, D, u, false, K, status, st);
     if (e != cudaSuccess) return e;
     return launch_gemv(packed, s, out, K, u, batch, o, status, st);  // a programmatic dependent of the lift
 }

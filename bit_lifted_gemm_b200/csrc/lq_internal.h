@@ -15,8 +15,17 @@ namespace lq {
 cudaError_t launch_pack(const int8_t* signs, int out, int K, uint32_t* packed, cudaStream_t st);
 cudaError_t launch_unpack(const uint32_t* packed, int out, int K, int8_t* signs, cudaStream_t st);
 
+// Activation lift u = blockdiag(M^T) T^{-1} a. `status` is the device status word
+// (the tensor-core prefill variant has bounded waits).
 cudaError_t launch_lift(const void* a, bool a_bf16, int batch, int in, const float* tinv, int tblk,
-                        const float* M, int d, int D, void* u, bool u_bf16, int K, cudaStream_t st);
+                        const float* M, int d, int D, void* u, bool u_bf16, int K, unsigned* status,
+                        cudaStream_t st);
+
+// Prefill lift with the whitening on tcgen05 (bf16 activations, 128-wide
+// whitening blocks, at least 64 tokens); launch_lift dispatches to it.
+bool lift_tc_supported(bool a_bf16, int batch, int in, const float* tinv, int tblk, int d, int D);
+cudaError_t launch_lift_tc(const uint16_t* a, int batch, int in, const float* tinv, const float* M, int d, int D,
+                           void* u, bool u_bf16, int K, unsigned* status, cudaStream_t st);
 
 // Decode GEMV (integer tensor cores; u quantized per CTA). `status` is the
 // device status word that bounded waits report to.

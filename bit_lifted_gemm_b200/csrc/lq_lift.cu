@@ -510,7 +510,10 @@ cudaError_t raise_smem_limit(const void* fn, size_t bytes, int which) {
 }  // namespace
 
 cudaError_t launch_lift(const void* a, bool a_bf16, int batch, int in, const float* tinv, int tblk,
-                        const float* M, int d, int D, void* u, bool u_bf16, int K, cudaStream_t st) {
+                        const float* M, int d, int D, void* u, bool u_bf16, int K, unsigned* status,
+                        cudaStream_t st) {
+    if (lift_tc_supported(a_bf16, batch, in, tinv, tblk, d, D))
+        return launch_lift_tc(static_cast<const uint16_t*>(a), batch, in, tinv, M, d, D, u, u_bf16, K, status, st);
     LiftArgs p;
     p.a = a; p.tinv = tinv; p.M = M; p.u = u;
     p.a_bf16 = a_bf16; p.u_bf16 = u_bf16;

@@ -111,6 +111,35 @@ def test_lift_padding_and_small_blocks(lq):
         assert rel_err(u, want) <= 1e-6
 
 
+@pytest.mark.parametrize("in_dim,d,D,batch,u_dtype", [
+    (5120, 10, 24, 200, "bf16"),  # LQ-24/10 channels: runs of 120 straddling 128-wide blocks, ragged tokens
+    (1024, 8, 20, 130, "f32"),    # runs aligned to the whitening blocks, fp32 output, 2-token last tile
+    (2048, 16, 40, 64, "bf16"),   # smallest batch of the tensor-core path
+    (1280, 20, 40, 300, "bf16"),  # d = 20: runs of 6 lift blocks
+    (384, 8, 9, 70, "bf16"),      # odd D (scalar stores), zero tail of 16 lifted entries
+    (384, 8, 9, 100, "f32"),      # same with fp32 output
+    (640, 5, 9, 128, "bf16"),     # d = 5: runs of 25 lift blocks (125 channels)
+])
+def test_lift_tensor_core_prefill(lq, in_dim, d, D, batch, u_dtype):
+    """Prefill lift with the whitening on tcgen05 (bf16 activations, 128-wide blocks)."""
+    from datagen.inputs import bf16_bits_from_f32
+    g = rng_for(62, in_dim, d * 1000 + batch)
+    a = bf16_bits_from_f32(g.standard_normal((batch, in_dim)).astype(np.float32))
+    M = (g.standard_normal((d, D)) / np.sqrt(D)).astype(np.float32)
+    tinv = (g.standard_normal((in_dim // 128, 128, 128)) / np.sqrt(128)).astype(np.float32)
+    K = oracle.lifted_dim(in_dim, d, D)
+    u = host(lq.lift_activations(dev(a), dev(M), K, tinv=dev(tinv), u_dtype=u_dtype))
+    want = oracle.lift(oracle.whiten(oracle.to_f64(a, "bf16"), oracle.to_f64(tinv)), oracle.to_f64(M), K)
+    kreal = (in_dim // d) * D
+    if u_dtype == "bf16":
+        u = oracle.to_f64(u, "bf16")
+        assert np.all(np.abs(u - want) <= _bf16_ulp(want) + 1e-6 * np.max(np.abs(want)))
+    else:
+        assert rel_err(u, want) <= 1e-6
+        assert np.max(np.abs(u - want)) <= 1e-5 * np.max(np.abs(want))
+    assert np.all(u[:, kreal:] == 0.0)
+
+
 @pytest.mark.parametrize("in_dim,d,D,tblk,batch,a_bf16,u_dtype", [
     (1024, 16, 48, 256, 3, True, "f32"),   # two float4 per lane of a T row, second M column per lane
     (960, 10, 40, 96, 2, False, "f32"),    # d-blocks straddling whitening blocks
