@@ -37,9 +37,9 @@
 //     same load whatever the shape. A tile is two 16-word steps of 16 rows
 //     (2 KB, one 3-D TMA box) when the row length allows, else one step. Each
 //     warp streams its tiles through a private ring, one mbarrier per stage,
-//     every wait bounded. A warp writes one exact partial per group it
-//     touches; the partials of a group are added in warp order: deterministic
-//     results.
+//     every wait bounded. A warp adds the exact integer total of each group it
+//     touches into the CTA's per-(group, column, row) sums with 64-bit shared
+//     atomics: integer addition, so the result does not depend on the order.
 //   * The GEMV is launched as a programmatic dependent of whatever precedes it
 //     on the stream (normally the activation lift): it requests its first
 //     weight tiles early and waits (griddepcontrol.wait) only before reading u.
@@ -66,6 +66,7 @@ constexpr int kStepWords = 16;    // words per row a warp consumes per step
 constexpr int kStepBytes = 16 * kStepWords * 4;  // one step of 16 rows x 64 bytes
 constexpr int kMaxRounds = 2;     // quantization items per thread kept in registers (staged path)
 constexpr int kUBoxRows = 16;     // words per TMA box of u
+constexpr int kWordsPerSweep = kThreads / 8;  // direct u path: eight threads per 32-element word
 constexpr int kMaxSegSteps = 255;  // steps one 32-bit segment sum holds
 constexpr size_t kSmemBudget = 220 * 1024;
 
@@ -129,24 +130,6 @@ __device__ __forceinline__ int max_exponent(unsigned cmax_bits) {
     return E == 0 ? -126 : E - 126;
 }
 
-// 32 elements of word x of a column of u from global memory (zeros past the end of K).
-__device__ __forceinline__ void load_word(const float* uc, int x, int kw, float (&v)[32]) {
-    if (x < kw) {
-        const float4* src = reinterpret_cast<const float4*>(uc + 32 * x);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float4 f = __ldg(src + q);
-            v[4 * q] = f.x;
-            v[4 * q + 1] = f.y;
-            v[4 * q + 2] = f.z;
-            v[4 * q + 3] = f.w;
-        }
-    } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0.f;
-    }
-}
-
 // 32 elements of staged row `row` (128 bytes, 128-byte swizzle: 16-byte chunk q
 // of row r sits at chunk q ^ (r & 7)), or zeros when !valid.
 __device__ __forceinline__ void read_staged(const uint8_t* stage, int row, bool valid, float (&v)[32]) {
@@ -191,6 +174,36 @@ __device__ __forceinline__ int word_digits(const float (&v)[32], float sa, float
     return (int)(bsum - 32u * kMagicBits);
 }
 
+// Elements j, j + 8, j + 16, j + 24 of word x of a column of u (zeros past the
+// end of K): the four bytes of one B register.
+__device__ __forceinline__ float4 load_quarter(const float* uc, int x, int kw, int j) {
+    if (x >= kw) return make_float4(0.f, 0.f, 0.f, 0.f);
+    const float* q = uc + 32 * x + j;
+    return make_float4(__ldg(q), __ldg(q + 8), __ldg(q + 16), __ldg(q + 24));
+}
+
+// Digits of four elements (j, j + 8, j + 16, j + 24 of a word): plane pl of
+// P[pl] in bytes 0..3. Returns their sum of u_q.
+__device__ __forceinline__ int quarter_digits(const float4& v, float sa, float sb, uint32_t (&P)[3]) {
+    const float e[4] = {v.x, v.y, v.z, v.w};
+    uint32_t tb[4];
+    uint32_t bsum = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t b = __float_as_uint(fmaf(e[i] * sa, sb, kRoundMagic));  // u_q = b - kMagicBits
+        bsum += b;
+        tb[i] = (b - (kMagicBits - 0x808080u)) ^ 0x808080u;  // (u_q + 0x808080) ^ 0x808080
+    }
+    const uint32_t t0 = __byte_perm(tb[0], tb[1], 0x5140);  // a0 b0 a1 b1
+    const uint32_t t1 = __byte_perm(tb[2], tb[3], 0x5140);  // c0 d0 c1 d1
+    const uint32_t t2 = __byte_perm(tb[0], tb[1], 0x0062);  // a2 b2 .  .
+    const uint32_t t3 = __byte_perm(tb[2], tb[3], 0x0062);  // c2 d2 .  .
+    P[0] = __byte_perm(t0, t1, 0x5410);
+    P[1] = __byte_perm(t0, t1, 0x7632);
+    P[2] = __byte_perm(t2, t3, 0x5410);
+    return (int)(bsum - 4u * kMagicBits);
+}
+
 struct GemvArgs {
     const uint32_t* packed;
     const float* s;
@@ -201,18 +214,18 @@ struct GemvArgs {
     int c0, ncols;    // columns [c0, c0 + ncols) in this pass (ncols <= 2)
     int kx0, kwc;     // words [kx0, kx0 + kwc) of K in this launch; kx0, kwc multiples of 16
     int ngroups;      // 16-row groups of the layer; CTA b owns [b*ngroups/grid, (b+1)*ngroups/grid)
-    int maxseg;       // partial-sum slots per warp
+    int maxgroups;    // most 16-row groups a CTA owns
     int pitch;        // chunks per shared-memory digit plane
     int accumulate;   // 1: o += this launch's result
 };
 
 // Shared-memory carve-up (offsets from a 1024-byte-aligned base).
 struct Layout {
-    size_t ring, work, zero, bars, part, sall, colmax, wbound, total;
+    size_t ring, work, zero, bars, gacc, sall, colmax, total;
 };
 
 __host__ __device__ inline Layout gemv_layout(int ts, int stages, bool tma, bool ustage, int ncols, int kwc,
-                                              int pitch, int maxseg) {
+                                              int pitch, int maxgroups) {
     Layout L;
     L.ring = 0;
     const size_t rings = tma ? (size_t)kWarps * stages * ts * kStepBytes : 0;
@@ -221,11 +234,10 @@ __host__ __device__ inline Layout gemv_layout(int ts, int stages, bool tma, bool
     const size_t staged = ustage ? (size_t)ncols * kwc * 128 : 0;
     L.zero = L.work + (((planes > staged ? planes : staged) + 127) & ~(size_t)127);
     L.bars = L.zero + 128;
-    L.part = L.bars + (size_t)kWarps * (stages + 1) * 8;
-    L.sall = L.part + (size_t)kWarps * maxseg * ncols * 16 * 8;
+    L.gacc = L.bars + (size_t)kWarps * (stages + 1) * 8;
+    L.sall = L.gacc + (size_t)maxgroups * ncols * 16 * 8;
     L.colmax = L.sall + kMaxColsPass * 8;
-    L.wbound = L.colmax + kMaxColsPass * 4;
-    L.total = L.wbound + (kWarps + 1) * 4 + 1024;  // + alignment slack
+    L.total = L.colmax + kMaxColsPass * 4 + 1024;  // + alignment slack
     return L;
 }
 
@@ -299,16 +311,17 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
     const int ndig = 3 * p.ncols;
     constexpr int kTileBytes = TS * kStepBytes;
 
-    const Layout L = gemv_layout(TS, STAGES, TMA, USTAGE, p.ncols, p.kwc, p.pitch, p.maxseg);
+    const Layout L = gemv_layout(TS, STAGES, TMA, USTAGE, p.ncols, p.kwc, p.pitch, p.maxgroups);
     uint8_t* ring = smem + L.ring + (size_t)warp * STAGES * kTileBytes;
     uint8_t* work = smem + L.work;
     uint4* bplanes = reinterpret_cast<uint4*>(work);
     uint4* bzero = reinterpret_cast<uint4*>(smem + L.zero);  // 8 zero chunks: digits of idle MMA columns
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars) + warp * (STAGES + 1);  // ring stages, then u
-    double* part = reinterpret_cast<double*>(smem + L.part);  // [warp][segment][column][16 rows]
+    // sum_{bit=1} u_q per (group, column, row), exact integers added with shared
+    // atomics (the same result in any order)
+    unsigned long long* gacc = reinterpret_cast<unsigned long long*>(smem + L.gacc);
     unsigned long long* sall = reinterpret_cast<unsigned long long*>(smem + L.sall);
     unsigned* colmax = reinterpret_cast<unsigned*>(smem + L.colmax);
-    int* wbound = reinterpret_cast<int*>(smem + L.wbound);  // warp w owns tiles [wbound[w], wbound[w+1])
     const uint32_t ubar = sm100::smem_addr(bars + STAGES);
 
     // Next tile to request (lane 0): ring index nxt, step xs of its group, row y.
@@ -354,7 +367,7 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
         colmax[threadIdx.x] = 0u;
         sall[threadIdx.x] = 0ull;
     }
-    if (threadIdx.x <= kWarps) wbound[threadIdx.x] = split_point(threadIdx.x, total, kWarps);
+    for (int i = threadIdx.x; i < (gend - gbeg) * p.ncols * 16; i += kThreads) gacc[i] = 0ull;
     __syncthreads();
 
     // u is written by the kernel before this one on the stream
@@ -365,6 +378,7 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
     // maxima, pass 2 writes the digit planes
     const int nitems = p.ncols * p.kwc;
     const int nrounds = (nitems + kThreads - 1) / kThreads;
+    const int jq = threadIdx.x & 7, wq = threadIdx.x >> 3;  // direct path: element group, word of the sweep
     float v[kMaxRounds][32];
     bool ufail = false;
     if constexpr (USTAGE) {
@@ -402,34 +416,77 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
             }
         }
     } else {
-        for (int rd = 0; rd < nrounds; ++rd) {
-            const int it = rd * kThreads + threadIdx.x;
-            const bool live = it < nitems;
-            const int c = live ? it / p.kwc : 0;
-            load_word(p.u + (long long)(p.c0 + c) * p.K, live ? p.kx0 + it - c * p.kwc : p.kw, p.kw, v[0]);
-            if (TMA && rd == 0 && lane == 0)
-                while (nxt < t1 && nxt < t0 + STAGES - 1) issue();
-            reduce_max(colmax, live, c, __float_as_uint(absmax32(v[0])), lane);
+        // u read directly, eight threads per word: thread jq of a word takes its
+        // elements jq, jq + 8, jq + 16, jq + 24. A warp's four words never cross a
+        // column (K chunks are multiples of 16 words). Four sweeps of 48 words
+        // are in flight at once.
+        if (TMA && lane == 0)
+            while (nxt < t1 && nxt < t0 + STAGES - 1) issue();
+        for (int w0 = 0; w0 < nitems; w0 += 4 * kWordsPerSweep) {
+            float4 q[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int it = w0 + k * kWordsPerSweep + wq;
+                const int c = it < nitems ? it / p.kwc : 0;
+                q[k] = load_quarter(p.u + (long long)(p.c0 + c) * p.K, it < nitems ? p.kx0 + it - c * p.kwc : p.kw,
+                                    p.kw, jq);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int it = w0 + k * kWordsPerSweep + wq;
+                const bool live = it < nitems;
+                const float mx = fmaxf(fmaxf(fabsf(q[k].x), fabsf(q[k].y)), fmaxf(fabsf(q[k].z), fabsf(q[k].w)));
+                reduce_max(colmax, live, live ? it / p.kwc : 0, __float_as_uint(mx), lane);
+            }
         }
     }
     __syncthreads();  // every staged word has been read: the planes may overwrite the staging area
+    if constexpr (USTAGE) {
 #pragma unroll
-    for (int rd = 0; rd < (USTAGE ? kMaxRounds : 1); ++rd) {
-        for (int r2 = rd; r2 < (USTAGE ? rd + 1 : nrounds); ++r2) {
-            if (USTAGE && r2 >= nrounds) break;
-            const int it = r2 * kThreads + threadIdx.x;
+        for (int rd = 0; rd < kMaxRounds; ++rd) {
+            if (rd >= nrounds) break;
+            const int it = rd * kThreads + threadIdx.x;
             const bool live = it < nitems;
             const int c = live ? it / p.kwc : 0;
             const int xl = it - c * p.kwc;
             int qsum = 0;
             if (live) {
-                if (!USTAGE && nrounds > 1) load_word(p.u + (long long)(p.c0 + c) * p.K, p.kx0 + xl, p.kw, v[0]);
                 const int F = 22 - max_exponent(colmax[c]);  // column max * 2^F < 2^22
                 uint32_t P[3][8];
                 qsum = word_digits(v[rd], pow2f(F >> 1), pow2f(F - (F >> 1)), P);
                 store_digits(bplanes, p.pitch, c, xl, P);
             }
             reduce_sum(sall, live, c, qsum, lane);
+        }
+    } else {
+        for (int w0 = 0; w0 < nitems; w0 += 4 * kWordsPerSweep) {
+            float4 q[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int it = w0 + k * kWordsPerSweep + wq;
+                const int c = it < nitems ? it / p.kwc : 0;
+                q[k] = load_quarter(p.u + (long long)(p.c0 + c) * p.K, it < nitems ? p.kx0 + it - c * p.kwc : p.kw,
+                                    p.kw, jq);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int it = w0 + k * kWordsPerSweep + wq;
+                const bool live = it < nitems;
+                const int c = live ? it / p.kwc : 0;
+                int qsum = 0;
+                if (live) {
+                    const int xl = it - c * p.kwc;
+                    const int F = 22 - max_exponent(colmax[c]);
+                    uint32_t P[3];
+                    qsum = quarter_digits(q[k], pow2f(F >> 1), pow2f(F - (F >> 1)), P);
+                    // element jq of word pair (xl & ~1): word 2 (jq >> 1) + (jq & 1) of its chunk run
+                    uint32_t* base = reinterpret_cast<uint32_t*>(bplanes + chunkpos(xl & ~1)) + (xl & 1) +
+                                     4 * (jq >> 1) + 2 * (jq & 1);
+#pragma unroll
+                    for (int pl = 0; pl < 3; ++pl) base[(size_t)(3 * c + pl) * p.pitch * 4] = P[pl];
+                }
+                reduce_sum(sall, live, c, qsum, lane);
+            }
         }
     }
     __syncthreads();
@@ -442,8 +499,7 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
     const uint32_t bar0 = sm100::smem_addr(bars);
     const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
     int kfail = -1;  // ring index whose wait ran out
-    int seg = 0;
-    for (int tt = t0; tt < t1; ++seg) {
+    for (int tt = t0; tt < t1;) {
         const int gl = tt / tpg;
         const int tend = min(t1, (gl + 1) * tpg);
         int acc[8][4];
@@ -490,8 +546,9 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
         }
         if (kfail >= 0) break;
         // ---- segment partial: V = sum_j 2^(7-j) acc_j = 2^7 sum_{bit=1} d per digit
-        // column (|V| < 2^23 per step, so 32 bits hold up to 255 steps); gather
-        // the three planes of each batch column with shuffles
+        // column (|V| < 2^23 per step, so 32 bits hold up to 255 steps); the three
+        // planes of each batch column are gathered with shuffles and sum_{bit=1}
+        // u_q is added into the CTA's per-(group, column, row) total
         int vreg[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -500,7 +557,7 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
             for (int j = 1; j < 8; ++j) vv = 2 * vv + acc[j][e];
             vreg[e] = vv;
         }
-        double* dst = part + (size_t)(warp * p.maxseg + seg) * p.ncols * 16;
+        unsigned long long* gdst = gacc + (size_t)gl * p.ncols * 16;
 #pragma unroll
         for (int c = 0; c < kMaxColsPass; ++c) {
             if (c >= p.ncols) break;
@@ -513,7 +570,7 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
                     const int vv = __shfl_sync(0xffffffffu, vreg[2 * hr + (col & 1)], (lane & ~3) | (col >> 1));
                     s1 += (long long)vv << (8 * pl);  // exact: 2^7 sum_{bit=1} u_q
                 }
-                if (t == 0) dst[c * 16 + g + 8 * hr] = (double)s1 * (1.0 / 64.0);  // 2 sum_{bit=1} u_q
+                if (t == 0) atomicAdd(gdst + c * 16 + g + 8 * hr, (unsigned long long)(s1 >> 7));
             }
         }
     }
@@ -527,21 +584,16 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
     }
     __syncthreads();
 
-    // ---- per (group, column, row): add the warps' partials in warp order, finish, store
+    // ---- per (group, column, row): finish and store
     const int nout = (gend - gbeg) * p.ncols * 16;
     for (int item = threadIdx.x; item < nout; item += kThreads) {
         const int row = item & 15, c = (item >> 4) % p.ncols, gl = (item >> 4) / p.ncols;
         const int m = m0 + 16 * gl + row;
         if (m >= p.out) continue;
-        double sum = 0.0;
-        for (int w = 0; w < kWarps; ++w) {
-            const int a = wbound[w], b = wbound[w + 1];
-            if (a < b && a < (gl + 1) * tpg && b > gl * tpg)  // empty ranges touch no group
-                sum += part[((size_t)(w * p.maxseg + (gl - a / tpg)) * p.ncols + c) * 16 + row];
-        }
         const int F = 22 - max_exponent(colmax[c]);
-        // sum_k sigma u_q = 2 sum_{bit=1} u_q - sum_k u_q, then undo the 2^F scale
-        const double val = (sum - (double)(long long)sall[c]) * __longlong_as_double((long long)(1023 - F) << 52);
+        // sum_k sigma u_q = 2 sum_{bit=1} u_q - sum_k u_q (exact integers), then undo the 2^F scale
+        const long long sig = 2 * (long long)gacc[item] - (long long)sall[c];
+        const double val = (double)sig * __longlong_as_double((long long)(1023 - F) << 52);
         float* out = p.o + (long long)(p.c0 + c) * p.out + m;
         const float res = (float)(val * (double)__ldg(p.s + m));
         *out = p.accumulate ? *out + res : res;
@@ -577,22 +629,15 @@ EncodeTiledFn encode_fn() {
 }
 
 struct Plan {
-    int grid, ts, stages, cols, kwc, pitch, maxseg;
+    int grid, ts, stages, cols, kwc, pitch, maxgroups;
     bool tma, ustage;
     size_t smem;
 };
 
-// Partial-sum slots a warp needs: the groups its tile range can touch.
-int max_segments(int grid, int ngroups, int tpg) {
-    const long long gmax = (ngroups + grid - 1) / grid;
-    const long long len = (gmax * tpg + kWarps - 1) / kWarps;
-    return (int)((len + tpg - 1) / tpg + 1);
-}
-
 // One CTA per SM (or per group when there are fewer groups). Preference: up to
 // two columns per pass, then a deep ring (three tiles in flight per warp), then
 // the widest K chunk whose digit planes fit in shared memory (a second launch
-// costs less than a shallow ring), then u staged by TMA.
+// costs less than a shallow ring: measured), then u staged by TMA.
 Plan make_plan(int out, int kw, int batch) {
     const int ngroups = (out + 15) / 16;
     Plan pl;
@@ -601,6 +646,7 @@ Plan make_plan(int out, int kw, int batch) {
     const int q = pl.ts * kStepWords;  // K chunks hold whole tiles (zeros past the row end)
     const int kwp = (kw + q - 1) / q * q;
     pl.grid = std::min(num_sms(), ngroups);
+    pl.maxgroups = (ngroups + pl.grid - 1) / pl.grid;
     for (int cols = std::min(kMaxColsPass, batch); cols >= 1; --cols) {
         pl.cols = cols;
         for (int deep = pl.tma ? 1 : 0; deep >= 0; --deep) {
@@ -609,16 +655,15 @@ Plan make_plan(int out, int kw, int batch) {
                 pl.kwc = ((kwp + nchunks - 1) / nchunks + q - 1) / q * q;
                 if (pl.kwc > kMaxSegSteps * kStepWords) continue;  // 32-bit segment sums
                 pl.pitch = plane_pitch(pl.kwc);
-                const int tpg = (pl.kwc / kStepWords + pl.ts - 1) / pl.ts;
-                pl.maxseg = max_segments(pl.grid, ngroups, tpg);
                 const int nrounds = (cols * pl.kwc + kThreads - 1) / kThreads;
                 for (int us = 1; us >= 0; --us) {
                     pl.ustage = us && pl.tma && nrounds <= kMaxRounds;
                     if (us && !pl.ustage) continue;
-                    pl.smem =
-                        gemv_layout(pl.ts, pl.stages, pl.tma, pl.ustage, cols, pl.kwc, pl.pitch, pl.maxseg).total;
+                    pl.smem = gemv_layout(pl.ts, pl.stages, pl.tma, pl.ustage, cols, pl.kwc, pl.pitch, pl.maxgroups)
+                                  .total;
                     if (pl.smem <= kSmemBudget) return pl;
                 }
+                if (pl.kwc == q) break;  // narrowest chunk already
             }
         }
     }
@@ -726,7 +771,7 @@ cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, 
             p.kx0 = kx0;
             p.kwc = pl.kwc;
             p.ngroups = (out + 15) / 16;
-            p.maxseg = pl.maxseg;
+            p.maxgroups = pl.maxgroups;
             p.pitch = pl.pitch;
             p.accumulate = kx0 > 0;
             cudaError_t e = launch_planned(wmap, umap, p, pl, st);

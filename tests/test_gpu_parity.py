@@ -184,7 +184,10 @@ def test_tiny_layer_full_path(lq, batch):
 
 
 @pytest.mark.parametrize("out,K,batch", [(1000, 1536, 1), (1000, 1536, 3), (33, 1632, 16), (1, 32, 1),
-                                         (4097, 20480, 2), (700, 16384 + 1024, 1)])
+                                         (4097, 20480, 2), (700, 16384 + 1024, 1),
+                                         # many two-column passes, K chunks, ragged rows
+                                         (1000, 3072, 5), (777, 4096, 6), (513, 2048, 8), (2000, 8192, 9),
+                                         (300, 20480, 11), (1500, 12288, 16)])
 def test_gemv_ragged_vs_oracle(lq, out, K, batch):
     packed = make_packed_random(out, K, 52, extra=K + out)
     s = rng_for(52, 1, out).uniform(0.01, 0.03, out).astype(np.float32)
@@ -200,6 +203,18 @@ def test_gemv_integer_inputs_exact(lq):
     packed = make_packed_random(out, K, 53)
     s = np.ones(out, dtype=np.float32)
     u = g.integers(-8, 9, size=(batch, K)).astype(np.float32)
+    o = host(lq.gemv(dev(packed), dev(s), dev(u)))
+    want = oracle.contract(packed, s, oracle.to_f64(u))
+    assert np.array_equal(o.astype(np.float64), want)
+
+
+@pytest.mark.parametrize("out,K,batch", [(513, 4096, 8), (1001, 6144, 16)])
+def test_gemv_integer_inputs_exact_wide(lq, out, K, batch):
+    """Integer-valued u through several two-column passes: every sum is exact."""
+    g = rng_for(53, 6, batch)
+    packed = make_packed_random(out, K, 53, extra=batch)
+    s = np.ones(out, dtype=np.float32)
+    u = g.integers(-100, 101, size=(batch, K)).astype(np.float32)
     o = host(lq.gemv(dev(packed), dev(s), dev(u)))
     want = oracle.contract(packed, s, oracle.to_f64(u))
     assert np.array_equal(o.astype(np.float64), want)
