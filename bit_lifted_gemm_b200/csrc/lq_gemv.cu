@@ -294,6 +294,10 @@ __device__ __forceinline__ float absmax32(const float (&v)[32]) {
 template <int TS, int STAGES, bool TMA, bool USTAGE>
 __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift beside it
     gemv_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap umap, const GemvArgs p) {
+    // a dependent launch (the next K chunk or column pass) may be scheduled as
+    // SMs free up; it reads u and o only after its own griddepcontrol.wait,
+    // which waits for this grid to complete
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned (the 128-byte swizzle of staged u); offsetting the array
     // itself keeps every derived pointer in the shared address space
