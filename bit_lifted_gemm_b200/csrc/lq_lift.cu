@@ -230,15 +230,28 @@ __global__ void __launch_bounds__(64) lift_warp_kernel(LiftArgs p) {
 }
 
 // Few registers per warp let a GEMV CTA become resident beside the lift's CTAs
-// (and start its prologue) while the lift runs.
+// (and start its prologue) while the lift runs. The lift is itself launched as
+// a programmatic dependent of the kernel before it: its CTAs may start (and
+// stream T^-1) while that kernel finishes, and wait for it before reading the
+// activations.
 template <int Q, int NTOK>
 void launch_warp_lift(const LiftArgs& p, int d, dim3 grid, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(64, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (d <= 8)
-        lift_warp_kernel<Q, NTOK, 8><<<grid, 64, 0, st>>>(p);
+        cudaLaunchKernelEx(&cfg, lift_warp_kernel<Q, NTOK, 8>, p);
     else if (d <= 12)
-        lift_warp_kernel<Q, NTOK, 12><<<grid, 64, 0, st>>>(p);
+        cudaLaunchKernelEx(&cfg, lift_warp_kernel<Q, NTOK, 12>, p);
     else
-        lift_warp_kernel<Q, NTOK, 16><<<grid, 64, 0, st>>>(p);
+        cudaLaunchKernelEx(&cfg, lift_warp_kernel<Q, NTOK, 16>, p);
 }
 
 // ---------------------------------------------------------------- prefill variant

@@ -86,6 +86,10 @@ __device__ __forceinline__ void lift_block(const LiftArgs& p, int blk, int lane)
             const int j = lane + 32 * h;
             mc[h][i] = i < p.d && j < p.D ? __ldg(p.M + i * p.D + j) : 0.f;
         }
+    // T^-1 and M do not depend on the kernel before this one; the activations
+    // (and the u it may still read) do: wait for it here when launched as a
+    // programmatic dependent (a no-op otherwise)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int ba = Q > 0 ? (c0 / p.tblk) * p.tblk : 0;            // whitening block of the first channel
     const int bb = Q > 0 ? ((c0 + p.d - 1) / p.tblk) * p.tblk : 0;  // ... and of the last (ba or the next one)
     for (int tb = 0; tb < p.batch; tb += NTOK) {
