@@ -283,13 +283,13 @@ def oracle_sample(cfg_name, budget_s, nthreads):
     u, _ = oracle.forward(L.packed[:64], L.s[:64], a, t, M, cfg.K, nthreads)
     dt = time.perf_counter() - t0
     rows = int(min(cfg.out, max(64, 64 * budget_s / max(dt, 1e-6))))
-    # whole passes over the sample, repeated while they fill under a third of the budget
+    # whole passes over the sample, repeated until they fill most of the budget
     reps, t0 = 0, time.perf_counter()
     while True:
         oracle.forward(L.packed[:rows], L.s[:rows], a, t, M, cfg.K, nthreads)
         reps += 1
         dt = time.perf_counter() - t0
-        if dt >= budget_s / 3 or dt / reps * (reps + 1) > budget_s:
+        if dt >= 0.8 * budget_s or dt / reps * (reps + 1) > budget_s:
             break
     gbs = reps * rows * cfg.K / 8 / dt / 1e9
     return gbs, dt, (f"{cfg_name}: whitening + lift + sign contraction of {rows} of {cfg.out} rows, batch 1, "
