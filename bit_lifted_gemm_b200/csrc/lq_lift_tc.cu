@@ -343,7 +343,6 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
         fence_barrier_init();
         prefetch_tensormap(&amap);
     }
-    for (int i = threadIdx.x; i < p.d * p.D; i += TC_THREADS) Ms[i] = __ldg(p.M + i);
     if (warp == 1) {
         tmem_alloc(smem_addr(tmem_slot), TC_N);
         tmem_relinquish();
@@ -368,6 +367,10 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
                 issued = kb + 1;
             }
             if (issued > 0) mbar_wait(afull, (issued - 1) & 1, status);  // leave no copy in flight
+        } else {
+            // M is needed only by the lift at the end: its load stays off the
+            // critical path (the barrier before the epilogue orders it)
+            for (int i = lane - 1; i < p.d * p.D; i += 31) Ms[i] = __ldg(p.M + i);
         }
     } else if (warp == 1) {
         if (lane == 0) {
