@@ -152,12 +152,16 @@ constexpr uint32_t kMagicBits = 0x4B400000u;
 
 // Digits of one word: P[pl][j] holds, in byte i, digit pl of element j + 8 i.
 // Returns sum_e u_q[e] (|sum| < 2^27).
+// ONE: the scale is the single float sa (column maxima above 2^-104; one
+// rounding multiply-add per element); else sa * sb in two exact steps.
+template <bool ONE>
 __device__ __forceinline__ int word_digits(const float (&v)[32], float sa, float sb, uint32_t (&P)[3][8]) {
     uint32_t tb[32];  // balanced digits of element e in bytes 0..2 of tb[e]
     uint32_t bsum = 0;
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
-        const uint32_t b = __float_as_uint(fmaf(v[e] * sa, sb, kRoundMagic));  // u_q = b - kMagicBits
+        const uint32_t b = __float_as_uint(ONE ? fmaf(v[e], sa, kRoundMagic)
+                                               : fmaf(v[e] * sa, sb, kRoundMagic));  // u_q = b - kMagicBits
         bsum += b;
         tb[e] = (b - (kMagicBits - 0x808080u)) ^ 0x808080u;  // (u_q + 0x808080) ^ 0x808080
     }
@@ -221,7 +225,7 @@ struct GemvArgs {
 
 // Shared-memory carve-up (offsets from a 1024-byte-aligned base).
 struct Layout {
-    size_t ring, work, zero, bars, gacc, sall, colmax, total;
+    size_t ring, work, zero, bars, gacc, sall, colmax, srow, total;
 };
 
 __host__ __device__ inline Layout gemv_layout(int ts, int stages, bool tma, bool ustage, int ncols, int kwc,
@@ -237,7 +241,8 @@ __host__ __device__ inline Layout gemv_layout(int ts, int stages, bool tma, bool
     L.gacc = L.bars + (size_t)kWarps * (stages + 1) * 8;
     L.sall = L.gacc + (size_t)maxgroups * ncols * 16 * 8;
     L.colmax = L.sall + kMaxColsPass * 8;
-    L.total = L.colmax + kMaxColsPass * 4 + 1024;  // + alignment slack
+    L.srow = L.colmax + kMaxColsPass * 4;
+    L.total = L.srow + (size_t)kThreads * 4 + 1024;  // + alignment slack
     return L;
 }
 
@@ -326,6 +331,7 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
     unsigned long long* gacc = reinterpret_cast<unsigned long long*>(smem + L.gacc);
     unsigned long long* sall = reinterpret_cast<unsigned long long*>(smem + L.sall);
     unsigned* colmax = reinterpret_cast<unsigned*>(smem + L.colmax);
+    float* srow = reinterpret_cast<float*>(smem + L.srow);  // s of this CTA's first kThreads rows
     const uint32_t ubar = sm100::smem_addr(bars + STAGES);
 
     // Next tile to request (lane 0): ring index nxt, step xs of its group, row y.
@@ -372,6 +378,11 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
         sall[threadIdx.x] = 0ull;
     }
     for (int i = threadIdx.x; i < (gend - gbeg) * p.ncols * 16; i += kThreads) gacc[i] = 0ull;
+    // s of this CTA's rows is a weight: requested now, stored to shared memory
+    // only before the first barrier of the quantization (its latency hides
+    // behind the dependency wait and the landing of u)
+    const int nrow = (gend - gbeg) * 16;
+    const float s_own = threadIdx.x < nrow && m0 + threadIdx.x < p.out ? __ldg(p.s + m0 + threadIdx.x) : 0.f;
     __syncthreads();
 
     // u is written by the kernel before this one on the stream
@@ -444,6 +455,7 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
             }
         }
     }
+    if (threadIdx.x < nrow) srow[threadIdx.x] = s_own;
     __syncthreads();  // every staged word has been read: the planes may overwrite the staging area
     if constexpr (USTAGE) {
 #pragma unroll
@@ -457,7 +469,11 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
             if (live) {
                 const int F = 22 - max_exponent(colmax[c]);  // column max * 2^F < 2^22
                 uint32_t P[3][8];
-                qsum = word_digits(v[rd], pow2f(F >> 1), pow2f(F - (F >> 1)), P);
+                // 2^F as one factor when it is a float, else as two exact halves
+                if (F <= 127)
+                    qsum = word_digits<true>(v[rd], pow2f(F), 1.0f, P);
+                else
+                    qsum = word_digits<false>(v[rd], pow2f(F >> 1), pow2f(F - (F >> 1)), P);
                 store_digits(bplanes, p.pitch, c, xl, P);
             }
             reduce_sum(sall, live, c, qsum, lane);
@@ -599,7 +615,8 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for the lift 
         const long long sig = 2 * (long long)gacc[item] - (long long)sall[c];
         const double val = (double)sig * __longlong_as_double((long long)(1023 - F) << 52);
         float* out = p.o + (long long)(p.c0 + c) * p.out + m;
-        const float res = (float)(val * (double)__ldg(p.s + m));
+        const float sr = 16 * gl + row < kThreads ? srow[16 * gl + row] : __ldg(p.s + m);
+        const float res = (float)(val * (double)sr);
         *out = p.accumulate ? *out + res : res;
     }
 }
