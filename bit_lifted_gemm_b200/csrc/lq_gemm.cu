@@ -36,6 +36,7 @@ using namespace sm100;
 
 constexpr int BM = 128, BK = 64, STAGES = 4;
 constexpr int A_STAGE = BM * BK * 2;   // 16 KB
+constexpr int A_COLS = BK / 2;         // TMEM columns of one A stage (two bf16 per 32-bit column)
 constexpr int THREADS = 192;
 constexpr int UNPACK_THREADS = 128;
 template <int BN>
@@ -43,6 +44,15 @@ struct Tile {
     static constexpr int B_STAGE = BN * BK * 2;  // 32 KB (BN 256) or 8 KB (BN 64)
     static constexpr int TMEM_COLS = BN;         // fp32 accumulator, 128 lanes x BN columns
     static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * (A_STAGE + B_STAGE) + 256;
+};
+// The variant for short token runs keeps the A stages in TMEM after the
+// accumulator (the unpackers store them with tcgen05.st; no A traffic through
+// shared memory): measured faster for 64-token tiles, slower for 256-token ones.
+template <int BN>
+struct TileTA {
+    static constexpr int A_COL = BN;
+    static constexpr int TMEM_COLS = BN + STAGES * A_COLS <= 256 ? 256 : 512;  // a power of two
+    static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * Tile<BN>::B_STAGE + 256;
 };
 
 // Expand 16 sign bits (bit i = element i of a k-run) into 8 bf16x2 words:
@@ -238,6 +248,195 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
+template <int BN>
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_kernel_ta(const __grid_constant__ CUtensorMap tmap_u, const uint32_t* __restrict__ packed,
+                const float* __restrict__ s, int out, int K, int tokens, float* __restrict__ o,
+                unsigned* status) {
+    constexpr int B_STAGE = Tile<BN>::B_STAGE, TMEM_COLS = TileTA<BN>::TMEM_COLS, A_COL = TileTA<BN>::A_COL;
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte aligned for the 128-byte swizzle; offsetting the array itself
+    // keeps derived pointers in the shared address space
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    uint8_t* sB = smem;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + STAGES), accf = smem_addr(bars + 2 * STAGES);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
+    // K split in gridDim.z (1 or 2) parts: this CTA takes k-blocks [kb_lo, kb_hi),
+    // the split on a multiple of 8 k-blocks (aligned 16-word groups of sign words)
+    const int nkb_all = (K + BK - 1) / BK;
+    const int kb_lo = blockIdx.z == 0 ? 0 : (int)((long long)blockIdx.z * nkb_all / gridDim.z) & ~7;
+    const int kb_hi = blockIdx.z + 1 == gridDim.z ? nkb_all : (int)((long long)(blockIdx.z + 1) * nkb_all / gridDim.z) & ~7;
+    const int nkb = kb_hi - kb_lo;
+    const bool split = gridDim.z > 1;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < STAGES; ++st) {
+            mbar_init(full0 + 8 * st, 1 + UNPACK_THREADS);
+            mbar_init(empty0 + 8 * st, 1);
+        }
+        mbar_init(accf, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tmap_u);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int st = kb % STAGES, round = kb / STAGES;
+                if (round > 0 && !mbar_wait(empty0 + 8 * st, (round - 1) & 1, status)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(full0 + 8 * st, B_STAGE);
+                tma_load_2d(smem_addr(sB + st * B_STAGE), &tmap_u, (kb_lo + kb) * BK, n0, full0 + 8 * st);
+                issued = kb + 1;
+            }
+            // Do not leave copies in flight: wait (bounded) for the last load of each stage.
+            for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
+                mbar_wait(full0 + 8 * (kb % STAGES), (kb / STAGES) & 1, status);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(BM, BN);
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int st = kb % STAGES, round = kb / STAGES;
+                if (!mbar_wait(full0 + 8 * st, round & 1, status)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_tmem = tmem + A_COL + st * A_COLS, b_base = smem_addr(sB + st * B_STAGE);
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)  // 16 k = 8 TMEM columns of A, 32 bytes of a B row
+                    umma_f16_tmem_a(tmem, a_tmem + kk * 8, smem_desc_sw128(b_base + kk * 32), idesc, (kb | kk) != 0);
+                umma_commit(empty0 + 8 * st);
+            }
+            umma_commit(accf);  // fires once every issued MMA has completed
+        }
+    } else {
+        // ---- unpack: thread `row` writes row `row` of every A stage into TMEM
+        // lane `row`; a warp may only reach its own lane quadrant (warp % 4)
+        const int row = 32 * (warp & 3) + lane;
+        const int kw = K >> 5;
+        const int grow = m0 + row < out ? m0 + row : out - 1;  // rows past `out` are computed but never stored
+        const uint32_t* prow = packed + (long long)grow * kw;
+        const uint32_t a_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + A_COL;
+        // The row's sign words arrive 8 k-steps (16 words) at a time, the next
+        // group requested before the current one is expanded, so the unpackers
+        // do not wait a memory round trip per k-step.
+        const bool vec = (kw & 3) == 0;  // 16-byte aligned rows
+        auto load16 = [&](int kg0, uint32_t (&w)[16]) {
+            if (vec && (kg0 & 1) == 0 && 2 * kg0 + 16 <= kw) {
+                const uint4* src = reinterpret_cast<const uint4*>(prow + 2 * kg0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 x = __ldg(src + q);
+                    w[4 * q] = x.x;
+                    w[4 * q + 1] = x.y;
+                    w[4 * q + 2] = x.z;
+                    w[4 * q + 3] = x.w;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) w[q] = 2 * kg0 + q < kw ? __ldg(prow + 2 * kg0 + q) : 0u;  // u is zero past K
+            }
+        };
+        uint32_t cur[16], nxt[16];
+        load16(kb_lo, cur);
+        // The store of a stage is waited for only after the next k-step has been
+        // expanded, so its latency overlaps that work.
+        uint32_t v[32];
+        bool stop = false;
+        int pending = -1;  // stage stored but not yet released to the MMA
+        for (int kb0 = 0; kb0 < nkb && !stop; kb0 += 8) {
+            if (kb0 + 8 < nkb) load16(kb_lo + kb0 + 8, nxt);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int kb = kb0 + kk;
+                if (kb >= nkb || stop) break;
+                const int st = kb % STAGES, round = kb / STAGES;
+                expand16(cur[2 * kk] & 0xFFFFu, v);
+                expand16(cur[2 * kk] >> 16, v + 8);
+                expand16(cur[2 * kk + 1] & 0xFFFFu, v + 16);
+                expand16(cur[2 * kk + 1] >> 16, v + 24);
+                if (pending >= 0) {  // release the previous stage
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(full0 + 8 * pending);
+                    pending = -1;
+                }
+                // tcgen05.st is warp-collective: the warp decides together
+                const bool free = round == 0 || mbar_wait(empty0 + 8 * st, (round - 1) & 1, status);
+                if (!__all_sync(0xffffffffu, free)) {
+                    *abort_flag = 1;
+                    stop = true;
+                    break;
+                }
+                // word j holds k-elements (2j, 2j+1): TMEM column j of the stage
+                tmem_st_32x32b_x32(a_lane + st * A_COLS, v);
+                pending = st;
+            }
+#pragma unroll
+            for (int q = 0; q < 16; ++q) cur[q] = nxt[q];
+        }
+        if (pending >= 0) {
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(full0 + 8 * pending);
+        }
+
+        // ---- epilogue: TMEM -> registers -> s[r] * acc -> o[t][r]
+        const bool done = mbar_wait(accf, 0, status);
+        tc_fence_after();
+        // tcgen05.ld is warp-collective: decide for the whole warp at once
+        if (__all_sync(0xffffffffu, done && !*abort_flag)) {
+            const int q = warp & 3;  // this warp's TMEM lane quadrant
+            const int m = m0 + q * 32 + lane;
+            const float sr = m < out ? __ldg(s + m) : 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + c0, v);
+                tmem_ld_wait();
+                if (m < out) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = n0 + c0 + j;
+                        if (n < tokens) {
+                            if (split)
+                                atomicAdd(o + (long long)n * out + m, sr * __uint_as_float(v[j]));
+                            else
+                                o[(long long)n * out + m] = sr * __uint_as_float(v[j]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -268,12 +467,15 @@ cudaError_t launch_tile(const uint32_t* packed, const float* s, int out, int K, 
                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    // 64-token tiles: A stages in TMEM; wider tiles: A stages in shared memory
+    constexpr bool kTA = BN <= 64;
+    auto kern = kTA ? gemm_kernel_ta<BN> : gemm_kernel<BN>;
+    constexpr size_t smem = kTA ? TileTA<BN>::SMEM_BYTES : Tile<BN>::SMEM_BYTES;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)Tile<BN>::SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
@@ -284,7 +486,7 @@ cudaError_t launch_tile(const uint32_t* packed, const float* s, int out, int K, 
         cudaError_t e = cudaMemsetAsync(o, 0, (size_t)tokens * out * sizeof(float), st);
         if (e != cudaSuccess) return e;
     }
-    gemm_kernel<BN><<<grid, THREADS, Tile<BN>::SMEM_BYTES, st>>>(map, packed, s, out, K, tokens, o, status);
+    kern<<<grid, THREADS, smem, st>>>(map, packed, s, out, K, tokens, o, status);
     return cudaGetLastError();
 }
 
