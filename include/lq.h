@@ -79,7 +79,13 @@ LQ_API int lq_unpack_signs(const uint32_t* packed, int out, int K, int8_t* signs
  *            round to nearest even); u[c][b*D + j] = sum_i M[i][j] a'[c][b*d + i]
  *            with a' = T^{-1} a; entries at (in/d)*D .. K-1 are written as 0
  *   K      : must equal lq_lifted_dim(in, d, D); batch >= 1
- * Accumulation is fp32. */
+ * Accumulation is fp32. For bf16 activations with 128-wide whitening blocks and
+ * at least 64 tokens the whitening runs on the tensor cores with T^{-1} split
+ * into three bf16 parts (24 significant bits, fp32 accumulation): the same
+ * accuracy class as the fp32 kernels. Bounded waits inside that kernel report
+ * LQ_ERR_TIMEOUT through lq_get_device_status. The decode kernel is launched as
+ * a programmatic dependent of the preceding kernel on the stream and waits for
+ * it before reading a. */
 LQ_API int lq_lift_activations(const void* a, int a_dtype, int batch, int in,
                         const float* tinv, int tblk,
                         const float* M, int d, int D,
