@@ -311,7 +311,9 @@ def test_fused_step_vs_oracle_alternating_layers(lq):
 # ------------------------------------------------------------------ prefill GEMM
 
 @pytest.mark.parametrize("out,K,tokens", [(300, 1536, 300), (128, 64, 256), (129, 1568, 7), (1, 32, 1),
-                                          (517, 4096 + 32, 513)])
+                                          (517, 4096 + 32, 513),
+                                          # 64-token tiles (A stages in TMEM): aligned and ragged rows, K split
+                                          (1000, 12288, 64), (77, 4096, 50)])
 def test_gemm_isolated_vs_oracle(lq, out, K, tokens):
     packed = make_packed_random(out, K, 55, extra=K + out)
     s = rng_for(55, 1, out).uniform(0.01, 0.03, out).astype(np.float32)
@@ -321,9 +323,12 @@ def test_gemm_isolated_vs_oracle(lq, out, K, tokens):
     assert rel_err(o, want) <= 1e-5
 
 
-def test_gemm_integer_inputs_exact(lq):
-    g = rng_for(56, 5)
-    out, K, tokens = 260, 2048, 300
+@pytest.mark.parametrize("tokens", [300, 64, 33])
+def test_gemm_integer_inputs_exact(lq, tokens):
+    """Integer-valued u: bit-exact for 256-token tiles (A in shared memory) and
+    64-token tiles (A in TMEM, K split in two)."""
+    g = rng_for(56, 5, tokens)
+    out, K = 260, 2048
     packed = make_packed_random(out, K, 56)
     s = np.ones(out, dtype=np.float32)
     from datagen import bf16_bits_from_f32
