@@ -22,7 +22,8 @@ weak and the value sums all ranks' bytes over the slowest rank's time.
 One JSON line is printed by rank 0; it carries the roofline of the dominant
 kernel (the GEMV, timed alone right after the step region), the end-to-end
 number (pinned-host activations in, output back to the host, inside the timed
-region), sampled SM clocks, the float64 oracle timed on the host cores, and
+region: zero-copy, the lift loading and the GEMV storing the host buffers, with
+the copy-engine variant beside it), sampled SM clocks, the float64 oracle timed on the host cores, and
 secondary results (prefill GEMM TFLOP/s, the LQ-20/8 batch sweep, the LQ-D/8
 bit-width sweep).
 """
@@ -214,6 +215,13 @@ class DecodeLayer:
         lq.lift_gemv(self.a[i], self.M, self.packed[i], self.s[i], c.K, tinv=self.tinv[i], u=self.u[i], out=self.o[i])
         if with_copies:
             self.o_host[i].copy_(self.o[i], non_blocking=True)
+
+    def step_zero_copy(self, i):
+        """Host buffers in and out, no copy-engine transfers: the lift loads a
+        from pinned host memory and the GEMV stores o there."""
+        lq, c = self.lq, self.cfg
+        lq.lift_gemv(self.a_host[i], self.M, self.packed[i], self.s[i], c.K, tinv=self.tinv[i], u=self.u[i],
+                     out=self.o_host[i])
 
     def gemv_only(self, i):
         self.lq.gemv(self.packed[i], self.s[i], self.u[i], out=self.o[i])
@@ -429,6 +437,8 @@ def main():
               for b in range(blocks)]
     g_e2e = [capture(torch, lambda i, b=b: layer.step(b * STEPS_PER_GRAPH + i, with_copies=True), STEPS_PER_GRAPH)
              for b in range(blocks)]
+    g_zc = [capture(torch, lambda i, b=b: layer.step_zero_copy(b * STEPS_PER_GRAPH + i), STEPS_PER_GRAPH)
+            for b in range(blocks)]
 
     def replay_steps(graphs, n):
         full, rem = divmod(n, STEPS_PER_GRAPH)
@@ -474,13 +484,23 @@ def main():
     e_steps = max(STEPS_PER_GRAPH, min(args.steps, 16000) // STEPS_PER_GRAPH * STEPS_PER_GRAPH)
     barrier(world, device)
     torch.cuda.synchronize()
-    e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e4.record(st)
-    for k in range(e_steps // STEPS_PER_GRAPH):
-        g_e2e[k % blocks].replay()
-    e5.record(st)
-    e5.synchronize()
-    ms_e2e = max_over_ranks(e4.elapsed_time(e5), world, device) / e_steps
+    def time_e2e(graphs):
+        barrier(world, device)
+        torch.cuda.synchronize()
+        e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e4.record(st)
+        for k in range(e_steps // STEPS_PER_GRAPH):
+            graphs[k % blocks].replay()
+        e5.record(st)
+        e5.synchronize()
+        return max_over_ranks(e4.elapsed_time(e5), world, device) / e_steps
+
+    ms_e2e_copies = time_e2e(g_e2e)
+    ms_e2e = time_e2e(g_zc)
+    torch.cuda.synchronize()
+    for i in (0, copies - 1):   # zero-copy output equals the device step's, bit for bit
+        if not torch.equal(layer.o_host[i], layer.o[i].cpu()):
+            raise RuntimeError(f"zero-copy step {i} differs from the device step")
 
     packed_bytes = layer.packed_bytes
     value = world * packed_bytes / (ms_per_step * 1e-3) / 1e9
@@ -501,7 +521,13 @@ def main():
         "e2e": {"value": world * packed_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": int(layer.a[0].numel() * layer.a[0].element_size()),
                 "d2h_bytes_per_step": int(layer.o[0].numel() * 4), "ms_per_step": ms_e2e,
-                "note": "CUDA-graph replay of: H2D activations, lq_lift_gemv (lift + GEMV), D2H output"},
+                "mode": "zero-copy",
+                "note": "CUDA-graph replay of lq_lift_gemv on pinned host buffers: the lift loads the "
+                        "activations and the GEMV stores the output across the host link",
+                "copy_engine": {"value": world * packed_bytes / (ms_e2e_copies * 1e-3) / 1e9,
+                                "ms_per_step": ms_e2e_copies,
+                                "note": "H2D copy of the activations, lq_lift_gemv on device buffers, "
+                                        "D2H copy of the output"}},
         "gpu_launches": launches,
         "clocks": clocks,
     }
@@ -530,7 +556,7 @@ def main():
         print(json.dumps(result), flush=True)
     if world > 1:
         import torch.distributed as dist
-        del g_full, g_single, g_gemv, g_e2e
+        del g_full, g_single, g_gemv, g_e2e, g_zc
         dist.destroy_process_group()
 
 

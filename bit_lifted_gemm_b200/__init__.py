@@ -145,10 +145,19 @@ def gemv(packed, s, u, out=None, stream=None):
     return out
 
 
+def _dev_or_pinned(t, name):
+    if not t.is_contiguous() or not (t.is_cuda or t.is_pinned()):
+        raise ValueError(f"{name} must be a contiguous CUDA tensor or pinned host tensor")
+    return t
+
+
 def lift_gemv(a, M, packed, s, K, tinv=None, u=None, out=None, stream=None):
-    """Fused decode step: a [batch][in] (float32 or bfloat16) -> (u fp32 [batch][K], o fp32 [batch][out])."""
+    """Fused decode step: a [batch][in] (float32 or bfloat16) -> (u fp32 [batch][K], o fp32 [batch][out]).
+
+    `a` and `out` may be pinned host tensors (zero-copy: the kernels read and
+    write them across the host link); everything else lives on the device."""
     import torch
-    _dev_tensor(a, "a")
+    _dev_or_pinned(a, "a")
     _dev_tensor(M, "M")
     _dev_tensor(packed, "packed")
     batch, in_dim = a.shape
@@ -156,9 +165,11 @@ def lift_gemv(a, M, packed, s, K, tinv=None, u=None, out=None, stream=None):
     rows = packed.shape[0]
     a_t = LQ_BF16 if a.dtype == torch.bfloat16 else LQ_F32
     if u is None:
-        u = torch.empty((batch, K), dtype=torch.float32, device=a.device)
+        u = torch.empty((batch, K), dtype=torch.float32, device=M.device)
     if out is None:
-        out = torch.empty((batch, rows), dtype=torch.float32, device=a.device)
+        out = torch.empty((batch, rows), dtype=torch.float32, device=M.device)
+    _dev_tensor(u, "u")
+    _dev_or_pinned(out, "out")
     tblk = 0 if tinv is None else int(tinv.shape[-1])
     if tinv is not None:
         _dev_tensor(tinv, "tinv")

@@ -1,5 +1,5 @@
 // C ABI of the LiftQuant layer (declared in include/lq.h). This file validates
-// arguments synchronously, before any CUDA call, and enqueues the kernels on
+// arguments synchronously, before any launch, and enqueues the kernels on
 // the caller's stream. The only device state it owns is one status word per
 // device (a module-scope __device__ variable), which bounded waits in the
 // kernels set when they give up.
@@ -18,6 +18,19 @@ constexpr int kMaxDevices = 64;
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? LQ_OK : LQ_ERR_CUDA; }
+
+// True if kernels may load and store through p as given: device or managed
+// memory, or page-locked host memory that unified addressing maps at the same
+// address. Pageable host memory and unknown pointers are refused.
+bool device_addressable(const void* p) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) return true;
+    return at.type == cudaMemoryTypeHost && at.devicePointer == p;
+}
 
 // Device address of the status word on the current device (looked up once per device).
 unsigned* status_word(int* err) {
@@ -134,6 +147,7 @@ int lq_lift_gemv(const void* a, int a_dtype, int batch, int in, const float* tin
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    if (!device_addressable(a) || !device_addressable(o)) return LQ_ERR_INVALID_ARG;
     int err = LQ_OK;
     unsigned* status = status_word(&err);
     if (!status) return err;

@@ -11,7 +11,8 @@
  * K = (in/d)*D rounded up to a multiple of 32, so the weight bit-width is D/d.
  *
  * Conventions shared by every call
- *  - All tensor pointers are caller-owned DEVICE memory, 16-byte aligned,
+ *  - All tensor pointers are caller-owned DEVICE memory (lq_lift_gemv's `a`
+ *    and `o` may also be mapped page-locked host memory), 16-byte aligned,
  *    densely packed row-major. The library frees nothing and keeps no pointer.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
  *    stream-ordered and asynchronous: they return after enqueueing work.
@@ -113,7 +114,16 @@ LQ_API int lq_gemv(const uint32_t* packed, const float* s, int out, int K,
  *   o : fp32 [batch][out] (written); 1 <= batch <= 16
  * Results are exactly those of the two calls; the GEMV is launched as a
  * programmatic dependent of the lift, so its setup and first weight requests
- * overlap the lift. Requires an sm_100 device (else LQ_ERR_UNSUPPORTED). */
+ * overlap the lift.
+ * Zero-copy decode: `a` and `o` (only these two) may instead be page-locked
+ * host memory that the device addresses at the same pointer (with unified
+ * addressing, any cudaHostAlloc / cudaMallocHost buffer). The lift then loads
+ * the activations, and the GEMV stores the outputs, across the host link
+ * itself, so a step from host buffers needs no separate copies; the results
+ * are identical. The call checks both pointers with cudaPointerGetAttributes
+ * and returns LQ_ERR_INVALID_ARG for pageable or unmapped host memory. The
+ * host must not touch `a` or `o` until the stream has passed the call.
+ * Requires an sm_100 device (else LQ_ERR_UNSUPPORTED). */
 LQ_API int lq_lift_gemv(const void* a, int a_dtype, int batch, int in, const float* tinv, int tblk,
                         const float* M, int d, int D, const uint32_t* packed, const float* s, int out, int K,
                         float* u, float* o, void* stream);

@@ -292,6 +292,50 @@ def test_fused_step_equals_two_calls(lq, name, batch):
     assert np.array_equal(host(o_f), host(o))
 
 
+def _pinned(x):
+    import torch
+    t = dev(x).cpu()
+    return t.pin_memory()
+
+
+@pytest.mark.parametrize("name,batch", [("tiny", 3), ("decode_lq24_10", 1), ("decode_lq20_8", 4),
+                                        ("decode_lq20_8", 16)])
+def test_fused_step_zero_copy(lq, name, batch):
+    """Activations read from, and outputs written to, pinned host memory by the
+    kernels themselves: identical to the all-device call (batch 16 also splits K
+    over launches, so the GEMV accumulates into host memory)."""
+    import torch
+    L = make_layer(CONFIGS[name], batch)
+    u_d, o_d = _fused(lq, L)
+    a_h = _pinned(L.a)
+    o_h = torch.full((batch, L.cfg.out), float("nan"), dtype=torch.float32).pin_memory()
+    t = None if L.tinv is None else dev(L.tinv)
+    u_z, o_z = lq.lift_gemv(a_h, dev(L.M), dev(L.packed), dev(L.s), L.cfg.K, tinv=t, out=o_h)
+    torch.cuda.synchronize()
+    assert o_z.data_ptr() == o_h.data_ptr()
+    assert np.array_equal(host(u_z), host(u_d))
+    assert np.array_equal(o_h.numpy(), host(o_d))
+
+
+def test_fused_step_rejects_pageable_host(lq):
+    """Pageable host memory is refused before any launch (binding and C ABI)."""
+    import ctypes
+    import torch
+    L = make_layer(CONFIGS["tiny"], 1)
+    a_p = torch.from_numpy(np.ascontiguousarray(L.a))
+    with pytest.raises(ValueError):
+        lq.lift_gemv(a_p, dev(L.M), dev(L.packed), dev(L.s), L.cfg.K)
+    u = torch.empty((1, L.cfg.K), dtype=torch.float32, device="cuda")
+    o = torch.empty((1, L.cfg.out), dtype=torch.float32, device="cuda")
+    M, pk, s = dev(L.M), dev(L.packed), dev(L.s)
+    d, D = L.M.shape
+    rc = lq.lib.lq_lift_gemv(ctypes.c_void_p(a_p.data_ptr()), lq.LQ_F32, 1, L.cfg.in_dim, None, 0,
+                             ctypes.c_void_p(M.data_ptr()), d, D, ctypes.c_void_p(pk.data_ptr()),
+                             ctypes.c_void_p(s.data_ptr()), L.cfg.out, L.cfg.K, ctypes.c_void_p(u.data_ptr()),
+                             ctypes.c_void_p(o.data_ptr()), None)
+    assert rc == lq.LQ_ERR_INVALID_ARG
+
+
 def test_fused_step_vs_oracle_alternating_layers(lq):
     """One-call decode step against the oracle, alternating a small and a large
     layer (32 and 148 CTAs)."""
