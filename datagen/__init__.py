@@ -8,10 +8,12 @@ sharing any computation.
 
 from .inputs import (  # noqa: F401
     CONFIGS,
+    KronFactors,
     LayerConfig,
     LayerInputs,
     bf16_bits_from_f32,
     f32_from_bf16_bits,
+    make_kron_factors,
     make_layer,
     make_signs_pm1,
     make_packed_random,

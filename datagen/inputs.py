@@ -6,14 +6,18 @@ re-drawn alone and the same bytes reach the oracle and the GPU path.
 
 Tensor ids: 0 = weight signs, 1 = row scales s, 2 = projection M,
 3 = whitening inverse blocks, 4 = activations a, 5 = lifted activations u
-drawn directly (used to isolate the contraction from the lift).
+drawn directly (used to isolate the contraction from the lift), 6 = factors
+of a Kronecker-factored whitening inverse.
 
 Distributions follow the synthetic workloads of the LiftQuant layer:
 signs iid Bernoulli(0.5); s ~ U[0.01, 0.03]; M ~ N(0, 1/D) in fp32;
 whitening-inverse blocks are random orthogonal 128x128 matrices (Q of a
 Householder QR of a Gaussian matrix, column signs fixed so diag(R) > 0,
 rounded to fp32); activations ~ N(0, 1) in fp32 or bf16 (round to nearest
-even).
+even). Kronecker factors of T^{-1} = diag(r2) (Q1 kron Q2) diag(r1): Q1, Q2 a
+random orthogonal matrix plus N(0, 0.05^2 / n) noise (learned factors start
+orthogonal and drift), r1 = exp(U[-0.5, 0.5]) per channel, r2 = exp(U[-0.25,
+0.25]) per d-block, all fp32.
 """
 
 from __future__ import annotations
@@ -26,7 +30,7 @@ import numpy as np
 BASE_SEED = 0x4C51
 
 # tensor stream ids
-SIGNS, SCALES, PROJ, TINV, ACT, LIFTED = 0, 1, 2, 3, 4, 5
+SIGNS, SCALES, PROJ, TINV, ACT, LIFTED, KRON = 0, 1, 2, 3, 4, 5, 6
 
 
 @dataclasses.dataclass(frozen=True)
@@ -120,6 +124,31 @@ def _orthogonal_blocks(nblk: int, tblk: int, g: np.random.Generator) -> np.ndarr
         q = q * np.sign(np.diag(r))[None, :]
         out[b] = q.astype(np.float32)
     return out
+
+
+@dataclasses.dataclass
+class KronFactors:
+    r1: np.ndarray   # fp32 [in]
+    q1: np.ndarray   # fp32 [n1][n1]
+    q2: np.ndarray   # fp32 [n2][n2]
+    r2: np.ndarray   # fp32 [in/d]
+
+
+def make_kron_factors(in_dim: int, n1: int, d: int, cfg_index: int, extra: int = 0) -> KronFactors:
+    """Seeded factors of a Kronecker-factored whitening inverse for in = n1 * n2."""
+    assert in_dim % n1 == 0 and in_dim % d == 0
+    n2 = in_dim // n1
+    g = rng_for(cfg_index, KRON, extra)
+
+    def factor(n):
+        q, r = np.linalg.qr(g.standard_normal((n, n)))
+        q = q * np.sign(np.diag(r))[None, :]
+        return (q + 0.05 / np.sqrt(n) * g.standard_normal((n, n))).astype(np.float32)
+
+    q1, q2 = factor(n1), factor(n2)
+    r1 = np.exp(g.uniform(-0.5, 0.5, in_dim)).astype(np.float32)
+    r2 = np.exp(g.uniform(-0.25, 0.25, in_dim // d)).astype(np.float32)
+    return KronFactors(r1, q1, q2, r2)
 
 
 @dataclasses.dataclass

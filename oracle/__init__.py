@@ -12,6 +12,8 @@ Parity status of each routine (what pins it, in tests/test_oracle_pins.py):
   lifted_dim       closed form K = (in/d)*D, bit-width K/in = D/d
   pack/unpack      hand-derived golden words + round trip
   whiten           identity, permutation (brute force), norm invariance
+  whiten_kron      Sylvester Hadamard H_n1 kron H_n2 = H_n (scipy), round trip
+                   T (T^{-1} a) = a with T built by numpy's kron, diagonal case
   lift             one-hot inputs recover M's rows at the right block; M = I
   contract         textbook +-1 GEMV (numpy matmul) when D = d, M = I, T = I;
                    exact integer brute force; bit-flip and negation identities
@@ -46,6 +48,7 @@ def _load():
         lib.lqo_pack_signs.argtypes = [_p, _i64, _i64, _p]
         lib.lqo_unpack_signs.argtypes = [_p, _i64, _i64, _p]
         lib.lqo_whiten.argtypes = [_p, _i64, _i64, _p, _i64, _p]
+        lib.lqo_whiten_kron.argtypes = [_p, _i64, _i64, _p, _p, _i64, _p, _i64, _p, _i64, _p]
         lib.lqo_lift.argtypes = [_p, _i64, _i64, _p, _int, _int, _i64, _p]
         lib.lqo_contract.argtypes = [_p, _p, _i64, _i64, _p, _i64, _p, _int]
         lib.lqo_contract_rows.argtypes = [_p, _p, _i64, _i64, _p, _i64, _p, _i64, _p]
@@ -100,6 +103,25 @@ def whiten(a: np.ndarray, tinv: Optional[np.ndarray]) -> np.ndarray:
     tblk = 0 if t is None else t.shape[-1]
     ap = np.zeros_like(a)
     _load().lqo_whiten(_ptr(a), batch, in_dim, _ptr(t), tblk, _ptr(ap))
+    return ap
+
+
+def whiten_kron(a: np.ndarray, r1: Optional[np.ndarray], q1: np.ndarray, q2: np.ndarray,
+                r2: Optional[np.ndarray], d: int) -> np.ndarray:
+    """a' = diag(r2) (Q1 kron Q2) diag(r1) a, r2 constant per d-block ([in/d] entries)."""
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    batch, in_dim = a.shape
+    q1 = np.ascontiguousarray(q1, dtype=np.float64)
+    q2 = np.ascontiguousarray(q2, dtype=np.float64)
+    n1, n2 = q1.shape[0], q2.shape[0]
+    assert q1.shape == (n1, n1) and q2.shape == (n2, n2) and n1 * n2 == in_dim and in_dim % d == 0
+    r1 = None if r1 is None else np.ascontiguousarray(r1, dtype=np.float64)
+    r2 = None if r2 is None else np.ascontiguousarray(r2, dtype=np.float64)
+    assert r1 is None or r1.shape == (in_dim,)
+    assert r2 is None or r2.shape == (in_dim // d,)
+    ap = np.zeros_like(a)
+    _load().lqo_whiten_kron(_ptr(a), batch, in_dim, _ptr(r1), _ptr(q1), n1, _ptr(q2), n2, _ptr(r2), d,
+                            _ptr(ap))
     return ap
 
 

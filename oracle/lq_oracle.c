@@ -87,6 +87,29 @@ void lqo_whiten(const double* a, int64_t batch, int64_t in, const double* tinv, 
     }
 }
 
+/* Kronecker-factored whitening (design 3: T = diag(s1) (P1 kron P2) diag(s2), with s2
+ * constant over each d-block), applied through the factors of its inverse
+ *   T^{-1} = diag(r2) (Q1 kron Q2) diag(r1),  r1 = 1/s1, Q1 = P1^{-1}, Q2 = P2^{-1}, r2 = 1/s2.
+ * in = n1 * n2. Kronecker entry (i, j) with i = i1*n2 + i2, j = j1*n2 + j2 is
+ * Q1[i1][j1] * Q2[i2][j2], so
+ *   a'[c][i] = r2[i / d] * sum_j Q1[i/n2][j/n2] * Q2[i%n2][j%n2] * r1[j] * a[c][j].
+ * r1 == NULL or r2 == NULL means all ones. O(in^2) per token: the definition, not a
+ * fast transform. */
+void lqo_whiten_kron(const double* a, int64_t batch, int64_t in, const double* r1, const double* q1,
+                     int64_t n1, const double* q2, int64_t n2, const double* r2, int64_t d, double* ap) {
+    for (int64_t c = 0; c < batch; ++c)
+        for (int64_t i = 0; i < in; ++i) {
+            const int64_t i1 = i / n2, i2 = i % n2;
+            double acc = 0.0;
+            for (int64_t j = 0; j < in; ++j) {
+                const int64_t j1 = j / n2, j2 = j % n2;
+                const double x = (r1 ? r1[j] : 1.0) * a[c * in + j];
+                acc += q1[i1 * n1 + j1] * q2[i2 * n2 + j2] * x;
+            }
+            ap[c * in + i] = (r2 ? r2[i / d] : 1.0) * acc;
+        }
+}
+
 /* Lift: u[c][blk*D+j] = sum_{i<d} M[i][j] a'[c][blk*d+i]; entries past (in/d)*D are 0.
  * This is M^T applied per d-block, i.e. the small matmul T* a of design 4, read
  * through w_i = sum_j M_ij y_j of design 1. */

@@ -118,6 +118,64 @@ def test_whiten_orthogonal_norm():
 
 # ---------------------------------------------------------------- lift
 
+# ------------------------------------------- Kronecker-factored whitening
+# T = diag(s1) (P1 kron P2) diag(s2), s2 constant per d-block (LiftQuant paper
+# note, "Key designs" 3); the oracle is handed the factors of T^{-1}.
+
+def test_whiten_kron_sylvester_hadamard():
+    """H_4 kron H_8 = H_32 in Sylvester's ordering, so normalised Hadamard
+    factors give the 32-point Walsh-Hadamard transform (scipy's matrix)."""
+    from scipy.linalg import hadamard
+    g = rng_for(90, 1, 0)
+    a = g.standard_normal((3, 32))
+    q1 = hadamard(4) / 2.0
+    q2 = hadamard(8) / np.sqrt(8.0)
+    got = oracle.whiten_kron(a, None, q1, q2, None, 4)
+    want = a @ (hadamard(32) / np.sqrt(32.0)).T
+    assert np.max(np.abs(got - want)) < 1e-13
+    assert np.allclose(np.linalg.norm(got, axis=1), np.linalg.norm(a, axis=1), rtol=1e-14)
+
+
+@pytest.mark.parametrize("n1,n2,d", [(3, 5, 5), (4, 6, 3), (2, 8, 4)])
+def test_whiten_kron_inverts_T(n1, n2, d):
+    """Round trip: T built densely from its factors with numpy's kron maps the
+    oracle's a' = T^{-1} a back to a. Catches swapped s1/s2, a transposed
+    factor, and the Kronecker index order (n1 != n2)."""
+    g = rng_for(90, 2, n1 * 100 + n2)
+    n = n1 * n2
+    p1 = g.standard_normal((n1, n1)) + 3 * np.eye(n1)
+    p2 = g.standard_normal((n2, n2)) + 3 * np.eye(n2)
+    s1 = np.exp(g.uniform(-1, 1, n))
+    s2_blk = np.exp(g.uniform(-1, 1, n // d))
+    T = np.diag(s1) @ np.kron(p1, p2) @ np.diag(np.repeat(s2_blk, d))
+    a = g.standard_normal((2, n))
+    ap = oracle.whiten_kron(a, 1.0 / s1, np.linalg.inv(p1), np.linalg.inv(p2), 1.0 / s2_blk, d)
+    assert np.max(np.abs(ap @ T.T - a)) < 1e-10
+
+
+def test_whiten_kron_diagonal_case():
+    """Identity factors: a' = r2[i/d] * r1[i] * a[i], element by element."""
+    g = rng_for(90, 3, 0)
+    n1, n2, d = 4, 10, 5
+    a = g.standard_normal((2, n1 * n2))
+    r1 = g.uniform(0.5, 2.0, n1 * n2)
+    r2 = g.uniform(0.5, 2.0, n1 * n2 // d)
+    got = oracle.whiten_kron(a, r1, np.eye(n1), np.eye(n2), r2, d)
+    assert np.array_equal(got, a * r1[None, :] * np.repeat(r2, d)[None, :])
+
+
+def test_whiten_kron_single_factor_is_block_whitening():
+    """Q1 = I: Q1 kron Q2 is block-diagonal with n1 copies of Q2, i.e. the
+    block whitening with tblk = n2 and every block equal to Q2."""
+    g = rng_for(90, 4, 0)
+    n1, n2 = 3, 8
+    q2 = g.standard_normal((n2, n2))
+    a = g.standard_normal((2, n1 * n2))
+    got = oracle.whiten_kron(a, None, np.eye(n1), q2, None, 4)
+    want = oracle.whiten(a, np.stack([q2] * n1))
+    assert np.max(np.abs(got - want)) < 1e-13
+
+
 def test_lift_one_hot_recovers_rows_of_M():
     g = rng_for(99, 2)
     d, D, nblk = 3, 7, 4
