@@ -356,6 +356,61 @@ def bench_decode_sweep(torch, lq, name, batches, l2, reps=50):
     return res
 
 
+def bench_kron(torch, lq, l2, reps=50):
+    """LQ-24/10 with the Kronecker-factored whitening (64 x 80 factors of T^-1):
+    the decode lift alone and lift + GEMV at batch 1 (weights rotating as in the
+    main step), and the lift of a 2048-token prefill (L2 flushed before each)."""
+    from datagen import make_kron_factors
+    cfg = CONFIGS["decode_lq24_10"]
+    dev = torch.device("cuda")
+    kf = make_kron_factors(cfg.in_dim, 64, cfg.d, cfg.index)
+    q1, q2, r1, r2 = (torch.from_numpy(x).to(dev) for x in (kf.q1, kf.q2, kf.r1, kf.r2))
+    layer = DecodeLayer(lq, cfg, 1, copies_for(cfg.out * cfg.K // 8, l2), torch)
+
+    def lift(i):
+        lq.lift_activations_kron(layer.a[i], q1, q2, layer.M, cfg.K, r1=r1, r2=r2, out=layer.u[i])
+
+    def step(i):
+        lift(i)
+        layer.gemv_only(i)
+
+    g_l = capture(torch, lift, STEPS_PER_GRAPH)
+    g_s = capture(torch, step, STEPS_PER_GRAPH)
+    for _ in range(3):
+        g_s.replay()
+    ms_lift = time_graph(torch, g_l, reps, STEPS_PER_GRAPH)
+    ms_step = time_graph(torch, g_s, reps, STEPS_PER_GRAPH)
+    del g_l, g_s, layer
+
+    tokens = 2048
+    L = make_layer(CONFIGS["prefill_lq24_10"], tokens, packed=False)
+    a = torch.from_numpy(L.a.view(np.int16)).to(dev).view(torch.bfloat16)
+    M = torch.from_numpy(L.M).to(dev)
+    u = torch.empty((tokens, cfg.K), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(int(400e6) // 4, dtype=torch.float32, device=dev)
+    st = torch.cuda.current_stream()
+    for _ in range(3):
+        lq.lift_activations_kron(a, q1, q2, M, cfg.K, r1=r1, r2=r2, u_dtype="bf16", out=u)
+    times = []
+    for _ in range(10):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        lq.lift_activations_kron(a, q1, q2, M, cfg.K, r1=r1, r2=r2, u_dtype="bf16", out=u)
+        e1.record(st)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms_pre = float(np.median(times))
+    n1, n2 = kf.q1.shape[0], kf.q2.shape[0]
+    flop_tok = 2 * cfg.in_dim * (n1 + n2) + 2 * cfg.in_dim // cfg.d * cfg.d * cfg.D
+    del flush, u, a
+    torch.cuda.empty_cache()
+    return {"factors": f"{n1}x{n1} and {n2}x{n2}",
+            "decode_b1": {"lift_us": ms_lift * 1e3, "step_us": ms_step * 1e3,
+                          "step_GBps": cfg.out * cfg.K // 8 / (ms_step * 1e-3) / 1e9},
+            "prefill_2048": {"lift_us": ms_pre * 1e3, "lift_TFLOPs": tokens * flop_tok / (ms_pre * 1e-3) / 1e12}}
+
+
 def bench_prefill(torch, lq, name, tokens, reps=10):
     cfg = CONFIGS[name]
     L = make_layer(cfg, tokens)
@@ -542,6 +597,7 @@ def main():
             n = f"sweep_lq{D}_8"
             extra[n] = {"b1": bench_decode_sweep(torch, lq, n, (1,), l2)["1"],
                         "b64": bench_prefill(torch, lq, n, 64)}
+        extra["kron_lq24_10"] = bench_kron(torch, lq, l2)
         result["extra"] = extra
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -23,7 +23,7 @@ LQ_OK, LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_TIMEOUT = 0, 
 LQ_F32, LQ_BF16 = 0, 1
 
 SYMBOLS = ("lq_status_str", "lq_lifted_dim", "lq_pack_signs", "lq_unpack_signs", "lq_lift_activations",
-           "lq_gemv", "lq_lift_gemv", "lq_gemm", "lq_get_device_status")
+           "lq_lift_activations_kron", "lq_gemv", "lq_lift_gemv", "lq_gemm", "lq_get_device_status")
 
 
 class LQError(RuntimeError):
@@ -47,6 +47,8 @@ def _load() -> ctypes.CDLL:
     lib.lq_unpack_signs.argtypes = [p, i, i, p, p]
     lib.lq_lift_activations.restype = i
     lib.lq_lift_activations.argtypes = [p, i, i, i, p, i, p, i, i, p, i, i, p]
+    lib.lq_lift_activations_kron.restype = i
+    lib.lq_lift_activations_kron.argtypes = [p, i, i, i, p, p, i, p, i, p, p, i, i, p, i, i, p]
     lib.lq_gemv.restype = i
     lib.lq_gemv.argtypes = [p, p, i, i, p, i, p, p]
     lib.lq_lift_gemv.restype = i
@@ -129,6 +131,29 @@ def lift_activations(a, M, K, tinv=None, u_dtype="f32", out=None, stream=None):
         _dev_tensor(tinv, "tinv")
     _check(lib.lq_lift_activations(_ptr(a), a_t, batch, in_dim, _ptr(tinv), tblk, _ptr(M), d, D, _ptr(out), u_t,
                                    K, _stream(stream)), "lq_lift_activations")
+    return out
+
+
+def lift_activations_kron(a, q1, q2, M, K, r1=None, r2=None, u_dtype="f32", out=None, stream=None):
+    """Lift with the Kronecker-factored whitening a' = diag(r2) (q1 kron q2) diag(r1) a.
+
+    a [batch][in] (float32 or bfloat16), q1 [n1][n1], q2 [n2][n2] with in = n1 * n2,
+    r1 [in] or None, r2 [in/d] or None -> u [batch][K] (float32 or bfloat16)."""
+    import torch
+    for t, name in ((a, "a"), (q1, "q1"), (q2, "q2"), (M, "M")):
+        _dev_tensor(t, name)
+    for t, name in ((r1, "r1"), (r2, "r2")):
+        if t is not None:
+            _dev_tensor(t, name)
+    batch, in_dim = a.shape
+    d, D = M.shape
+    a_t = LQ_BF16 if a.dtype == torch.bfloat16 else LQ_F32
+    u_t = LQ_BF16 if u_dtype in ("bf16", torch.bfloat16) else LQ_F32
+    if out is None:
+        out = torch.empty((batch, K), dtype=torch.bfloat16 if u_t == LQ_BF16 else torch.float32, device=a.device)
+    _check(lib.lq_lift_activations_kron(_ptr(a), a_t, batch, in_dim, _ptr(r1), _ptr(q1), int(q1.shape[0]), _ptr(q2),
+                                        int(q2.shape[0]), _ptr(r2), _ptr(M), d, D, _ptr(out), u_t, K,
+                                        _stream(stream)), "lq_lift_activations_kron")
     return out
 
 

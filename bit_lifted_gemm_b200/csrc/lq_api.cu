@@ -118,6 +118,27 @@ int lq_lift_activations(const void* a, int a_dtype, int batch, int in, const flo
                                      K, status, static_cast<cudaStream_t>(stream)));
 }
 
+int lq_lift_activations_kron(const void* a, int a_dtype, int batch, int in, const float* r1, const float* q1,
+                             int n1, const float* q2, int n2, const float* r2, const float* M, int d, int D,
+                             void* u, int u_dtype, int K, void* stream) {
+    if (!a || !q1 || !q2 || !M || !u) return LQ_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(q1) || !aligned16(q2) || !aligned16(M) || !aligned16(u))
+        return LQ_ERR_INVALID_ARG;
+    if ((r1 && !aligned16(r1)) || (r2 && !aligned16(r2))) return LQ_ERR_INVALID_ARG;
+    if ((a_dtype != LQ_F32 && a_dtype != LQ_BF16) || (u_dtype != LQ_F32 && u_dtype != LQ_BF16))
+        return LQ_ERR_INVALID_ARG;
+    if (batch < 1 || in < 1 || in > 16384 || d < 1 || d > 64 || D < 1 || D > 256 || d * D > 4096)
+        return LQ_ERR_INVALID_ARG;
+    if (n1 < 1 || n1 > 256 || n2 < 1 || n2 > 128 || n1 * n2 != in || in % d != 0) return LQ_ERR_INVALID_ARG;
+    if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
+    if (!lq::lift_kron_supported(batch, in, n1, n2, d, D)) return LQ_ERR_INVALID_ARG;
+    const int sm = is_sm100();
+    if (sm < 0) return LQ_ERR_CUDA;
+    if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    return from_cuda(lq::launch_lift_kron(a, a_dtype == LQ_BF16, batch, in, r1, q1, n1, q2, n2, r2, M, d, D, u,
+                                          u_dtype == LQ_BF16, K, static_cast<cudaStream_t>(stream)));
+}
+
 int lq_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u, int batch, float* o,
             void* stream) {
     if (!packed || !s || !u || !o) return LQ_ERR_INVALID_ARG;

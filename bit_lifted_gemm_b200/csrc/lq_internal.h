@@ -27,6 +27,14 @@ bool lift_tc_supported(bool a_bf16, int batch, int in, const float* tinv, int tb
 cudaError_t launch_lift_tc(const uint16_t* a, int batch, int in, const float* tinv, const float* M, int d, int D,
                            void* u, bool u_bf16, int K, unsigned* status, cudaStream_t st);
 
+// Lift with a Kronecker-factored whitening T^{-1} = diag(r2) (Q1 kron Q2) diag(r1)
+// (one thread-block cluster per token group, distributed shared memory).
+// lift_kron_supported tells whether the shapes fit its shared-memory plan.
+bool lift_kron_supported(int batch, int in, int n1, int n2, int d, int D);
+cudaError_t launch_lift_kron(const void* a, bool a_bf16, int batch, int in, const float* r1, const float* q1,
+                             int n1, const float* q2, int n2, const float* r2, const float* M, int d, int D,
+                             void* u, bool u_bf16, int K, cudaStream_t st);
+
 // Decode GEMV (integer tensor cores; u quantized per CTA). `status` is the
 // device status word that bounded waits report to.
 cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u,

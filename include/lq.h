@@ -92,6 +92,30 @@ LQ_API int lq_lift_activations(const void* a, int a_dtype, int batch, int in,
                         const float* M, int d, int D,
                         void* u, int u_dtype, int K, void* stream);
 
+/* Activation lift with the Kronecker-factored whitening of "Key designs" 3:
+ * T = diag(s1) (P1 kron P2) diag(s2) with s2 constant over each d-block, so
+ *   a' = T^{-1} a = diag(r2) (Q1 kron Q2) diag(r1) a,  r = 1/s, Q = P^{-1},
+ * and then u as in lq_lift_activations (s2 is thereby folded into the lift).
+ * The caller hands over the factors of T^{-1}; nothing is inverted here.
+ *   a      : [batch][in], a_dtype LQ_F32 or LQ_BF16; in = n1 * n2 <= 16384
+ *   r1     : fp32 [in] (1/s1), or NULL for ones
+ *   q1     : fp32 [n1][n1] (P1^{-1}), 1 <= n1 <= 256
+ *   q2     : fp32 [n2][n2] (P2^{-1}), 1 <= n2 <= 128
+ *   r2     : fp32 [in/d] (1/s2 of each d-block), or NULL for ones
+ *   M, d, D, u, u_dtype, K : as lq_lift_activations (in % d == 0)
+ * Kronecker entry ((i1, i2), (j1, j2)) is q1[i1][j1] * q2[i2][j2] with channel
+ * i = i1 * n2 + i2, so for one token, X = a reshaped row-major to n1 x n2,
+ * (Q1 kron Q2) x = Q1 X Q2^T: in * (n1 + n2) multiply-adds, fp32 throughout.
+ * Runs as thread-block clusters (no scratch memory); shapes whose
+ * shared-memory plan does not fit (e.g. a large odd n1) return
+ * LQ_ERR_INVALID_ARG. Launched as a programmatic dependent of the preceding
+ * kernel; it reads a only after that kernel completes. Requires an sm_100
+ * device (else LQ_ERR_UNSUPPORTED). */
+LQ_API int lq_lift_activations_kron(const void* a, int a_dtype, int batch, int in,
+                                    const float* r1, const float* q1, int n1, const float* q2, int n2,
+                                    const float* r2, const float* M, int d, int D,
+                                    void* u, int u_dtype, int K, void* stream);
+
 /* Decode 1-bit GEMV, batch 1..16 ("1-bit x float standard GEMM", "Key designs" 4):
  *   o[c][r] = s[r] * sum_k sigma[r][k] * u[c][k],  sigma = +1 if bit set else -1
  *   packed : uint32 [out][K/32]; s : fp32 [out]; u : fp32 [batch][K]

@@ -86,6 +86,20 @@ def _c(v):
     ("lift bad dtype", "lq_lift_activations", [_c(P), 7, 1, 640, None, 0, _c(P), 10, 24, _c(P), 0, 1536, None]),
     ("lift d too big", "lq_lift_activations", [_c(P), 0, 1, 130, None, 0, _c(P), 65, 2, _c(P), 0, 32, None]),
     ("lift batch 0", "lq_lift_activations", [_c(P), 0, 0, 640, None, 0, _c(P), 10, 24, _c(P), 0, 1536, None]),
+    ("kron n1*n2 != in", "lq_lift_activations_kron", [_c(P), 0, 1, 640, None, _c(P), 8, _c(P), 81, None, _c(P), 10,
+                                                      24, _c(P), 0, 1536, None]),
+    ("kron null q2", "lq_lift_activations_kron", [_c(P), 0, 1, 640, None, _c(P), 8, None, 80, None, _c(P), 10, 24,
+                                                  _c(P), 0, 1536, None]),
+    ("kron misaligned r1", "lq_lift_activations_kron", [_c(P), 0, 1, 640, _c(MIS), _c(P), 8, _c(P), 80, None, _c(P),
+                                                        10, 24, _c(P), 0, 1536, None]),
+    ("kron n2 too big", "lq_lift_activations_kron", [_c(P), 0, 1, 640, None, _c(P), 4, _c(P), 160, None, _c(P), 10,
+                                                     24, _c(P), 0, 1536, None]),
+    ("kron K mismatch", "lq_lift_activations_kron", [_c(P), 0, 1, 640, None, _c(P), 8, _c(P), 80, None, _c(P), 10,
+                                                     24, _c(P), 0, 1504, None]),
+    ("kron in too big", "lq_lift_activations_kron", [_c(P), 0, 1, 20480, None, _c(P), 160, _c(P), 128, None, _c(P),
+                                                     10, 24, _c(P), 0, 49152, None]),
+    ("kron plan too big (odd n1)", "lq_lift_activations_kron", [_c(P), 0, 1, 16320, None, _c(P), 255, _c(P), 64,
+                                                                None, _c(P), 10, 24, _c(P), 0, 39168, None]),
 ], ids=lambda c: c[0])
 def test_invalid_arguments_rejected_before_launch(case):
     import bit_lifted_gemm_b200 as lq

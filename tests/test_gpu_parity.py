@@ -272,6 +272,66 @@ def test_sweep_decode_sampled_rows(lq, D):
     assert rel_err(o[:, rows], want) <= 1e-5
 
 
+# ------------------------------------------------------------------ Kronecker-factored whitening
+
+def _kron_case(in_dim, n1, d, D, batch, a_dtype, seed):
+    from datagen import make_kron_factors
+    from datagen.inputs import bf16_bits_from_f32
+    g = rng_for(61, seed, batch)
+    a32 = g.standard_normal((batch, in_dim)).astype(np.float32)
+    a = bf16_bits_from_f32(a32) if a_dtype == "bf16" else a32
+    M = (g.standard_normal((d, D)) / np.sqrt(D)).astype(np.float32)
+    kf = make_kron_factors(in_dim, n1, d, 61, seed)
+    return a, M, kf
+
+
+def _kron_oracle_u(a, a_dtype, M, kf, d, K, with_r=True):
+    ap = oracle.whiten_kron(oracle.to_f64(a, a_dtype), oracle.to_f64(kf.r1) if with_r else None,
+                            oracle.to_f64(kf.q1), oracle.to_f64(kf.q2), oracle.to_f64(kf.r2) if with_r else None, d)
+    return oracle.lift(ap, oracle.to_f64(M), K)
+
+
+@pytest.mark.parametrize("in_dim,n1,d,D,batch,a_dtype,u_dtype,with_r", [
+    (640, 8, 10, 24, 1, "f32", "f32", True),      # clusters of 8 CTAs, one row of X each (padded to two)
+    (640, 8, 10, 24, 3, "f32", "f32", False),     # no diagonal factors
+    (5120, 64, 10, 24, 1, "bf16", "f32", True),   # LQ-24/10 decode layer, 64 x 80 factors
+    (5120, 64, 10, 24, 16, "bf16", "f32", True),
+    (8192, 64, 8, 20, 2, "bf16", "f32", True),    # LQ-20/8 layer, 64 x 128 factors
+    (70, 7, 5, 18, 2, "f32", "f32", True),        # odd n1: one CTA per token; n2 = 10 padded; K tail of 4
+    (48, 8, 4, 8, 3, "f32", "f32", True),         # d-blocks straddle rows of X; clusters of 4
+    (640, 8, 10, 24, 70, "bf16", "bf16", True),   # 4 tokens per cluster, ragged last cluster, bf16 output
+    (5120, 64, 10, 24, 40, "bf16", "bf16", True), # prefill-sized batch on the LQ-24/10 layer
+])
+def test_lift_kron(lq, in_dim, n1, d, D, batch, a_dtype, u_dtype, with_r):
+    """Lift with T^{-1} = diag(r2) (Q1 kron Q2) diag(r1) against the oracle."""
+    K = oracle.lifted_dim(in_dim, d, D)
+    a, M, kf = _kron_case(in_dim, n1, d, D, batch, a_dtype, 1)
+    u = host(lq.lift_activations_kron(dev(a), dev(kf.q1), dev(kf.q2), dev(M), K,
+                                      r1=dev(kf.r1) if with_r else None, r2=dev(kf.r2) if with_r else None,
+                                      u_dtype=u_dtype))
+    want = _kron_oracle_u(a, a_dtype, M, kf, d, K, with_r)
+    if u_dtype == "bf16":
+        u = oracle.to_f64(u, "bf16")
+        assert np.all(np.abs(u - want) <= _bf16_ulp(want) + 1e-6 * np.max(np.abs(want)))
+    else:
+        assert rel_err(u, want) <= 1e-6
+        assert np.max(np.abs(u - want)) <= 1e-5 * np.max(np.abs(want))
+    k0 = in_dim // d * D
+    assert np.all(u[:, k0:] == 0.0)
+
+
+def test_lift_kron_then_gemv_vs_oracle(lq):
+    """LQ-24/10 decode step with the Kronecker whitening: lift, then the GEMV."""
+    L = make_layer(CONFIGS["decode_lq24_10"], 1)
+    K = L.cfg.K
+    a, M, kf = _kron_case(L.cfg.in_dim, 64, L.cfg.d, L.cfg.D, 1, "bf16", 2)
+    u = lq.lift_activations_kron(dev(a), dev(kf.q1), dev(kf.q2), dev(M), K, r1=dev(kf.r1), r2=dev(kf.r2))
+    o = host(lq.gemv(dev(L.packed), dev(L.s), u))
+    rows = _sample_rows(L.cfg.out, 512, 11)
+    want = oracle.contract_rows(L.packed, L.s, _kron_oracle_u(a, "bf16", M, kf, L.cfg.d, K), rows)
+    assert rel_err(o[:, rows], want) <= 1e-5
+
+
 # ------------------------------------------------------------------ one-call decode step
 
 def _fused(lq, L):
