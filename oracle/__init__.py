@@ -19,6 +19,10 @@ Parity status of each routine (what pins it, in tests/test_oracle_pins.py):
                    exact integer brute force; bit-flip and negation identities
   dense_route      equals the lifted route (w.a' = y^T(M^T a'))
   codebook moments closed forms 0 and M M^T over all 2^D patterns
+  encode (brute)   M = I gives sign(w); local optimality against every one-bit
+                   flip; exact codewords M y* return y* with zero error
+  encode (search)  never below the brute-force optimum; exact codewords M y*
+                   recovered; D = d reduces to the closed form sign(M^{-1} w)
 """
 
 from __future__ import annotations
@@ -57,6 +61,7 @@ def _load():
         lib.lqo_forward.argtypes = [_p, _p, _i64, _i64, _p, _i64, _i64, _p, _i64, _p, _int, _int,
                                     _p, _p, _int]
         lib.lqo_codebook_moments.argtypes = [_p, _int, _int, _p, _p]
+        lib.lqo_encode_blocks.argtypes = [_p, _int, _int, _p, _i64, _int, _p, _p, _int]
         lib.lqo_block_identity_maxerr.restype = ctypes.c_double
         lib.lqo_block_identity_maxerr.argtypes = [_p, _int, _int, _p]
         _lib = lib
@@ -191,6 +196,29 @@ def forward(packed: np.ndarray, s: np.ndarray, a: np.ndarray, tinv: Optional[np.
                              _ptr(M), d, D, _ptr(u), _ptr(o), nthreads)
     assert rc == 0
     return u, o
+
+
+def encode_blocks(M: np.ndarray, w: np.ndarray, brute: bool = False,
+                  nthreads: int = 1) -> Tuple[np.ndarray, np.ndarray]:
+    """Blocks w [n][d] -> (sign patterns uint64 [n], bit j set <=> y_j = +1; squared
+    errors ||w - M y||^2 [n]). brute=True enumerates all 2^D patterns; otherwise the
+    pseudo-inverse start plus the 2^{D-d} auxiliary-vector search."""
+    M = np.ascontiguousarray(M, dtype=np.float64)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    d, D = M.shape
+    assert w.ndim == 2 and w.shape[1] == d and D <= 63 and D >= d
+    n = w.shape[0]
+    y = np.zeros(n, dtype=np.uint64)
+    err = np.zeros(n, dtype=np.float64)
+    _load().lqo_encode_blocks(_ptr(M), d, D, _ptr(w), n, int(brute), _ptr(y), _ptr(err), nthreads)
+    return y, err
+
+
+def patterns_to_signs(y: np.ndarray, D: int) -> np.ndarray:
+    """Sign patterns uint64 [n] -> +-1 int8 [n][D] (bit j set <=> +1)."""
+    y = np.asarray(y, dtype=np.uint64)
+    bits = (y[:, None] >> np.arange(D, dtype=np.uint64)[None, :]) & np.uint64(1)
+    return (2 * bits.astype(np.int8) - 1).astype(np.int8)
 
 
 def codebook_moments(M: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:

@@ -20,7 +20,7 @@ def build(force: bool = False) -> str:
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-Wall", "-Wextra",
-           "-o", tmp, SRC]
+           "-o", tmp, SRC, "-lm"]
     subprocess.check_call(cmd)
     os.replace(tmp, LIB)
     return LIB

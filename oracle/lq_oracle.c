@@ -14,7 +14,11 @@
  *   - a weight block w in R^d is represented as w ~= M y with y in {+-1}^D,
  *     M in R^{d x D}, so that w_i = sum_j M_ij y_j  (design 1);
  *   - storage is D sign bits per d weights, bit-width D/d  (design 1);
- *   - the whitening T acts on the activation side  (design 3);
+ *   - the whitening T acts on the activation side; in its Kronecker form
+ *     T = diag(s1)(P1 kron P2)diag(s2), s2 constant per block  (design 3);
+ *   - encoding a block means finding the nearest lifted codeword M y, which a
+ *     pseudo-inverse start plus a 2^{D-d} search over an auxiliary vector
+ *     approximates  (design 2);
  *   - at inference the decode matrix T* = M T^{-1} is applied to the
  *     activations once, followed by a 1-bit x float matmul with W_q and the
  *     per-row scale diag(s)  (design 4).
@@ -30,6 +34,7 @@
  * Every routine is a direct loop over its definition, in float64, with no
  * blocking, fusion or reordering.
  */
+#include <math.h>
 #include <pthread.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -273,4 +278,172 @@ double lqo_block_identity_maxerr(const double* M, int d, int D, const double* ap
     }
     free(mt);
     return worst;
+}
+
+/* ---------------------------------------------------------------- encoder
+ * "Key designs" 2: quantising a block w of d weights means finding the nearest
+ * point M y of the lifted codebook, y in {+-1}^D. Sign patterns are bit masks:
+ * bit j set <=> y_j = +1. Errors are squared Euclidean distances ||w - M y||^2. */
+
+static double lqo_code_err(const double* M, int d, int D, const double* w, uint64_t y) {
+    double e = 0.0;
+    for (int i = 0; i < d; ++i) {
+        double acc = w[i];
+        for (int j = 0; j < D; ++j) acc -= M[i * D + j] * (((y >> j) & 1u) ? 1.0 : -1.0);
+        e += acc * acc;
+    }
+    return e;
+}
+
+/* The naive search: all 2^D patterns; the lowest pattern wins a tie. */
+uint64_t lqo_encode_brute(const double* M, int d, int D, const double* w, double* err) {
+    uint64_t best = 0;
+    double best_e = lqo_code_err(M, d, D, w, 0);
+    for (uint64_t y = 1; y < (1ull << D); ++y) {
+        const double e = lqo_code_err(M, d, D, w, y);
+        if (e < best_e) {
+            best_e = e;
+            best = y;
+        }
+    }
+    *err = best_e;
+    return best;
+}
+
+/* x = A^{-1} b for a small dense n x n A (row-major), by Gauss-Jordan elimination
+ * with partial pivoting on copies. Returns 0 when A is singular. */
+static int lqo_solve(const double* A_in, const double* b_in, int n, double* x) {
+    double* A = (double*)malloc(sizeof(double) * (size_t)n * n);
+    memcpy(A, A_in, sizeof(double) * (size_t)n * n);
+    memcpy(x, b_in, sizeof(double) * (size_t)n);
+    int ok = 1;
+    for (int c = 0; c < n && ok; ++c) {
+        int piv = c;
+        for (int r = c + 1; r < n; ++r)
+            if (fabs(A[r * n + c]) > fabs(A[piv * n + c])) piv = r;
+        if (A[piv * n + c] == 0.0) {
+            ok = 0;
+            break;
+        }
+        if (piv != c) {
+            for (int k = 0; k < n; ++k) {
+                const double t = A[c * n + k];
+                A[c * n + k] = A[piv * n + k];
+                A[piv * n + k] = t;
+            }
+            const double t = x[c];
+            x[c] = x[piv];
+            x[piv] = t;
+        }
+        for (int r = 0; r < n; ++r) {
+            if (r == c) continue;
+            const double f = A[r * n + c] / A[c * n + c];
+            if (f == 0.0) continue;
+            for (int k = c; k < n; ++k) A[r * n + k] -= f * A[c * n + k];
+            x[r] -= f * x[c];
+        }
+    }
+    if (ok)
+        for (int c = 0; c < n; ++c) x[c] /= A[c * n + c];
+    free(A);
+    return ok;
+}
+
+/* The search of "Key designs" 2 (a pseudo-inverse start, then an auxiliary
+ * vector that cuts the search from 2^D to 2^{D-d} patterns), read as:
+ *   candidate 0:      y = sign(M^+ w), M^+ w = M^T (M M^T)^{-1} w;
+ *   candidate 1 + p:  for p in [0, 2^{D-d}), the auxiliary vector z is the first
+ *                     D - d coordinates (z_a = +1 iff bit a of p is set) and the
+ *                     last d coordinates solve M_B y_B = w - M_A z, rounded:
+ *                     y_B = sign(M_B^{-1} (w - M_A z)).
+ * sign(0) = +1. Returns the candidate of smallest error, the earliest on ties;
+ * *err is its error. Returns UINT64_MAX with *err = -1 if M M^T or M_B is singular. */
+uint64_t lqo_encode_search(const double* M, int d, int D, const double* w, double* err) {
+    const int na = D - d;
+    double* G = (double*)malloc(sizeof(double) * (size_t)d * d);
+    double* t = (double*)malloc(sizeof(double) * (size_t)(d > D ? d : D));
+    double* rhs = (double*)malloc(sizeof(double) * (size_t)d);
+    uint64_t best = UINT64_MAX;
+    double best_e = -1.0;
+    /* candidate 0: the pseudo-inverse start */
+    for (int i = 0; i < d; ++i)
+        for (int k = 0; k < d; ++k) {
+            double acc = 0.0;
+            for (int j = 0; j < D; ++j) acc += M[i * D + j] * M[k * D + j];
+            G[i * d + k] = acc;
+        }
+    if (!lqo_solve(G, w, d, t)) goto done;
+    {
+        uint64_t y0 = 0;
+        for (int j = 0; j < D; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < d; ++i) acc += M[i * D + j] * t[i];
+            if (acc >= 0.0) y0 |= 1ull << j;
+        }
+        best = y0;
+        best_e = lqo_code_err(M, d, D, w, y0);
+    }
+    /* candidates 1 + p: M_B holds the last d columns of M */
+    for (int i = 0; i < d; ++i)
+        for (int k = 0; k < d; ++k) G[i * d + k] = M[i * D + na + k];
+    for (uint64_t p = 0; p < (1ull << na); ++p) {
+        for (int i = 0; i < d; ++i) {
+            double acc = w[i];
+            for (int a = 0; a < na; ++a) acc -= M[i * D + a] * (((p >> a) & 1u) ? 1.0 : -1.0);
+            rhs[i] = acc;
+        }
+        if (!lqo_solve(G, rhs, d, t)) {
+            best = UINT64_MAX;
+            best_e = -1.0;
+            goto done;
+        }
+        uint64_t y = p;
+        for (int k = 0; k < d; ++k)
+            if (t[k] >= 0.0) y |= 1ull << (na + k);
+        const double e = lqo_code_err(M, d, D, w, y);
+        if (e < best_e) {
+            best_e = e;
+            best = y;
+        }
+    }
+done:
+    free(G);
+    free(t);
+    free(rhs);
+    *err = best_e;
+    return best;
+}
+
+/* Blocks [nblocks][d] of w -> patterns and errors; brute != 0 selects the naive search. */
+typedef struct {
+    const double* M; int d, D; const double* w; int64_t b0, b1; int brute; uint64_t* y; double* err;
+} lqo_encode_job;
+
+static void* lqo_encode_worker(void* p) {
+    lqo_encode_job* j = (lqo_encode_job*)p;
+    for (int64_t b = j->b0; b < j->b1; ++b)
+        j->y[b] = j->brute ? lqo_encode_brute(j->M, j->d, j->D, j->w + b * j->d, j->err + b)
+                           : lqo_encode_search(j->M, j->d, j->D, j->w + b * j->d, j->err + b);
+    return NULL;
+}
+
+void lqo_encode_blocks(const double* M, int d, int D, const double* w, int64_t nblocks, int brute, uint64_t* y,
+                       double* err, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t th[256];
+    lqo_encode_job jobs[256];
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t].M = M;
+        jobs[t].d = d;
+        jobs[t].D = D;
+        jobs[t].w = w;
+        jobs[t].b0 = nblocks * t / nthreads;
+        jobs[t].b1 = nblocks * (t + 1) / nthreads;
+        jobs[t].brute = brute;
+        jobs[t].y = y;
+        jobs[t].err = err;
+        pthread_create(&th[t], NULL, lqo_encode_worker, &jobs[t]);
+    }
+    for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
 }

@@ -343,3 +343,82 @@ def test_contract_rows_and_threads_agree():
     assert np.array_equal(o, o4)
     rows = np.array([0, 5, 511, 100])
     assert np.array_equal(oracle.contract_rows(L.packed, L.s, u, rows), o[:, rows])
+
+
+# ---------------------------------------------------------------- encoder
+# Nearest lifted codeword M y, y in {+-1}^D, of a block w of d weights
+# (LiftQuant paper note, "Key designs" 2).
+
+def _np_err(M, w, y, D):
+    s = oracle.patterns_to_signs(np.asarray([y], dtype=np.uint64), D)[0].astype(np.float64)
+    return float(np.sum((w - M @ s) ** 2))
+
+
+def test_encode_brute_identity_projection():
+    """M = I: the nearest point of {+-1}^d to w is sign(w), coordinate by coordinate."""
+    g = rng_for(91, 1, 0)
+    d = 8
+    w = g.standard_normal((20, d))
+    y, err = oracle.encode_blocks(np.eye(d), w, brute=True)
+    want = ((w >= 0).astype(np.uint64) << np.arange(d, dtype=np.uint64)[None, :]).sum(axis=1)
+    assert np.array_equal(y, want.astype(np.uint64))
+    assert np.allclose(err, np.sum((np.abs(w) - 1.0) ** 2, axis=1), rtol=1e-12, atol=1e-12)
+
+
+def test_encode_brute_locally_optimal():
+    """The brute-force optimum is at least as good as each of its D one-bit
+    neighbours, and its reported error is ||w - M y||^2 recomputed by numpy."""
+    g = rng_for(91, 2, 0)
+    d, D = 3, 9
+    M = g.standard_normal((d, D)) / np.sqrt(D)
+    w = g.standard_normal((15, d))
+    y, err = oracle.encode_blocks(M, w, brute=True)
+    for b in range(w.shape[0]):
+        e0 = _np_err(M, w[b], int(y[b]), D)
+        assert abs(e0 - err[b]) <= 1e-12 * max(1.0, e0)
+        for j in range(D):
+            assert _np_err(M, w[b], int(y[b]) ^ (1 << j), D) >= e0 - 1e-12
+
+
+@pytest.mark.parametrize("d,D", [(4, 10), (6, 14), (10, 16)])
+def test_encode_exact_codewords(d, D):
+    """w = M y*: both searches return y* with zero error (the auxiliary vector
+    z = y*_A makes the solved coordinates exact)."""
+    g = rng_for(91, 3, d * 100 + D)
+    M = g.standard_normal((d, D)) / np.sqrt(D)
+    ystar = g.integers(0, 1 << D, size=12, dtype=np.uint64)
+    w = oracle.patterns_to_signs(ystar, D).astype(np.float64) @ M.T
+    for brute in (True, False):
+        if brute and D > 14:
+            continue
+        y, err = oracle.encode_blocks(M, w, brute=brute)
+        assert np.array_equal(y, ystar)
+        assert np.all(err < 1e-20)
+
+
+@pytest.mark.parametrize("d,D", [(2, 8), (4, 12), (5, 13), (6, 14)])
+def test_encode_search_never_beats_brute(d, D):
+    g = rng_for(91, 4, d * 100 + D)
+    M = g.standard_normal((d, D)) / np.sqrt(D)
+    w = g.standard_normal((25, d))
+    _, eb = oracle.encode_blocks(M, w, brute=True)
+    ys, es = oracle.encode_blocks(M, w)
+    assert np.all(es >= eb - 1e-12)
+    for b in range(w.shape[0]):
+        assert abs(_np_err(M, w[b], int(ys[b]), D) - es[b]) <= 1e-12 * max(1.0, es[b])
+    # candidate 0 is the pseudo-inverse start, so no block ends worse than sign(M^+ w)
+    y0 = np.where(w @ np.linalg.pinv(M).T >= 0, 1.0, -1.0)
+    e0 = np.sum((w - y0 @ M.T) ** 2, axis=1)
+    assert np.all(es <= e0 + 1e-12)
+
+
+def test_encode_search_square_closed_form():
+    """D = d: no auxiliary coordinates, so the result is sign(M^{-1} w)."""
+    g = rng_for(91, 5, 0)
+    d = 6
+    M = g.standard_normal((d, d)) + 2 * np.eye(d)
+    w = g.standard_normal((10, d))
+    y, _ = oracle.encode_blocks(M, w)
+    x = np.linalg.solve(M, w.T).T
+    want = ((x >= 0).astype(np.uint64) << np.arange(d, dtype=np.uint64)[None, :]).sum(axis=1)
+    assert np.array_equal(y, want.astype(np.uint64))
