@@ -411,6 +411,31 @@ def bench_kron(torch, lq, l2, reps=50):
             "prefill_2048": {"lift_us": ms_pre * 1e3, "lift_TFLOPs": tokens * flop_tok / (ms_pre * 1e-3) / 1e12}}
 
 
+def bench_encode(torch, lq):
+    """Encoder (offline): seconds per million weights for LQ-24/10, LQ-16/8 and
+    LQ-32/16 on seeded Gaussian weights and projections, each sample sized to a
+    second or two (the cost per block grows as 2^(D-d))."""
+    dev = torch.device("cuda")
+    res = {}
+    for name, d, D, rows, in_dim in (("lq24_10", 10, 24, 26, 5120), ("lq16_8", 8, 16, 256, 4096),
+                                     ("lq32_16", 16, 32, 32, 4096)):
+        g = np.random.default_rng(0x4C51 + D)
+        M = torch.from_numpy((g.standard_normal((d, D)) / np.sqrt(D)).astype(np.float32)).to(dev)
+        w = torch.from_numpy(g.standard_normal((rows, in_dim)).astype(np.float32)).to(dev)
+        K = lq.lifted_dim(in_dim, d, D)
+        lq.encode(w[:1, :d * 64].contiguous(), M, lq.lifted_dim(d * 64, d, D))  # load the module
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        lq.encode(w, M, K)
+        e1.record()
+        e1.synchronize()
+        sec = e0.elapsed_time(e1) * 1e-3
+        res[name] = {"weights": rows * in_dim, "seconds": sec, "seconds_per_1M_weights": sec / (rows * in_dim) * 1e6,
+                     "patterns_per_block": 1 + 2 ** (D - d)}
+    return res
+
+
 def bench_prefill(torch, lq, name, tokens, reps=10):
     cfg = CONFIGS[name]
     L = make_layer(cfg, tokens)
@@ -598,6 +623,7 @@ def main():
             extra[n] = {"b1": bench_decode_sweep(torch, lq, n, (1,), l2)["1"],
                         "b64": bench_prefill(torch, lq, n, 64)}
         extra["kron_lq24_10"] = bench_kron(torch, lq, l2)
+        extra["encode"] = bench_encode(torch, lq)
         result["extra"] = extra
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -23,7 +23,8 @@ LQ_OK, LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_TIMEOUT = 0, 
 LQ_F32, LQ_BF16 = 0, 1
 
 SYMBOLS = ("lq_status_str", "lq_lifted_dim", "lq_pack_signs", "lq_unpack_signs", "lq_lift_activations",
-           "lq_lift_activations_kron", "lq_gemv", "lq_lift_gemv", "lq_gemm", "lq_get_device_status")
+           "lq_lift_activations_kron", "lq_gemv", "lq_lift_gemv", "lq_gemm", "lq_encode",
+           "lq_get_device_status")
 
 
 class LQError(RuntimeError):
@@ -54,6 +55,8 @@ def _load() -> ctypes.CDLL:
     lib.lq_lift_gemv.restype = i
     lib.lq_lift_gemv.argtypes = [p, i, i, i, p, i, p, i, i, p, p, i, i, p, p, p]
     lib.lq_gemm.restype = i
+    lib.lq_encode.restype = i
+    lib.lq_encode.argtypes = [p, i, i, p, i, i, p, i, p, p]
     lib.lq_gemm.argtypes = [p, p, i, i, p, i, p, p]
     lib.lq_get_device_status.restype = i
     lib.lq_get_device_status.argtypes = [p]
@@ -214,6 +217,22 @@ def gemm(packed, s, u, out=None, stream=None):
         out = torch.empty((tokens, rows), dtype=torch.float32, device=u.device)
     _check(lib.lq_gemm(_ptr(packed), _ptr(s), rows, K, _ptr(u), tokens, _ptr(out), _stream(stream)), "lq_gemm")
     return out
+
+
+def encode(w, M, K, err=False, out=None, stream=None):
+    """Encoder: weights w [rows][in] fp32, M [d][D] -> packed signs [rows][K/32]
+    (int32 storage of uint32), and the per-block squared errors [rows][in/d] when
+    err=True."""
+    import torch
+    _dev_tensor(w, "w")
+    _dev_tensor(M, "M")
+    rows, in_dim = w.shape
+    d, D = M.shape
+    if out is None:
+        out = torch.empty((rows, K // 32), dtype=torch.int32, device=w.device)
+    e = torch.empty((rows, in_dim // d), dtype=torch.float32, device=w.device) if err else None
+    _check(lib.lq_encode(_ptr(w), rows, in_dim, _ptr(M), d, D, _ptr(out), K, _ptr(e), _stream(stream)), "lq_encode")
+    return (out, e) if err else out
 
 
 def get_device_status(stream=None) -> int:

@@ -139,6 +139,20 @@ int lq_lift_activations_kron(const void* a, int a_dtype, int batch, int in, cons
                                           u_dtype == LQ_BF16, K, static_cast<cudaStream_t>(stream)));
 }
 
+int lq_encode(const float* w, int rows, int in, const float* M, int d, int D, uint32_t* packed, int K, float* err,
+              void* stream) {
+    if (!w || !M || !packed || !aligned16(w) || !aligned16(M) || !aligned16(packed)) return LQ_ERR_INVALID_ARG;
+    if (err && !aligned16(err)) return LQ_ERR_INVALID_ARG;
+    if (rows < 1 || in < 1 || d < 1 || d > 16 || D < d || D > 63 || D - d > 24 || in % d != 0)
+        return LQ_ERR_INVALID_ARG;
+    if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
+    if (lq::encode_smem(in, d, D) > 200 * 1024) return LQ_ERR_INVALID_ARG;
+    const int sm = is_sm100();
+    if (sm < 0) return LQ_ERR_CUDA;
+    if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    return from_cuda(lq::launch_encode(w, rows, in, M, d, D, packed, K, err, static_cast<cudaStream_t>(stream)));
+}
+
 int lq_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u, int batch, float* o,
             void* stream) {
     if (!packed || !s || !u || !o) return LQ_ERR_INVALID_ARG;

@@ -35,6 +35,13 @@ cudaError_t launch_lift_kron(const void* a, bool a_bf16, int batch, int in, cons
                              int n1, const float* q2, int n2, const float* r2, const float* M, int d, int D,
                              void* u, bool u_bf16, int K, cudaStream_t st);
 
+// Encoder (offline): nearest lifted codewords of weight blocks by the
+// pseudo-inverse start plus the 2^{D-d} auxiliary-vector search, float64,
+// written as packed signs. encode_smem gives its shared-memory need.
+size_t encode_smem(int in, int d, int D);
+cudaError_t launch_encode(const float* w, int rows, int in, const float* M, int d, int D, uint32_t* packed, int K,
+                          float* err, cudaStream_t st);
+
 // Decode GEMV (integer tensor cores; u quantized per CTA). `status` is the
 // device status word that bounded waits report to.
 cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u,

@@ -68,6 +68,28 @@ LQ_API int lq_pack_signs(const int8_t* signs_pm1, int out, int K, uint32_t* pack
 /* Inverse of lq_pack_signs: words -> int8 +-1 [out][K]. Bit-exact. */
 LQ_API int lq_unpack_signs(const uint32_t* packed, int out, int K, int8_t* signs_pm1, void* stream);
 
+/* Encoder, the offline step that produces W_q ("Key designs" 2): each block w
+ * of d consecutive weights of a row gets the sign pattern y in {+-1}^D whose
+ * codeword M y is (approximately) nearest, found as the page describes -- a
+ * pseudo-inverse start plus a search over an auxiliary vector that cuts the
+ * 2^D patterns to 2^{D-d}:
+ *   candidate 0:     y = sign(M^+ w), M^+ = M^T (M M^T)^{-1};
+ *   candidate 1 + p: the first D-d coordinates are the pattern p (bit a set
+ *                    <=> +1), the last d are sign(M_B^{-1} (w - M_A z)) with
+ *                    M_A, M_B the first D-d and last d columns of M;
+ *   sign(0) = +1; the smallest ||w - M y||^2 wins, the earliest on ties.
+ *   w      : fp32 [rows][in] (the weights to encode, already scaled/whitened)
+ *   M      : fp32 [d][D]; 1 <= d <= 16, d <= D <= 63, D - d <= 24, in % d == 0
+ *   packed : uint32 [rows][K/32] (written, the layout lq_gemv reads: block b of
+ *            a row occupies bits [b*D, (b+1)*D) of the lifted axis; padding 0)
+ *   K      : must equal lq_lifted_dim(in, d, D)
+ *   err    : fp32 [rows][in/d] squared errors ||w_blk - M y||^2, or NULL
+ * The search runs in float64 (its result is an integer code). If M M^T or M_B
+ * is singular every pattern is written as 0 and every err as NaN. Cost grows as
+ * 2^{D-d} per block. Requires an sm_100 device (else LQ_ERR_UNSUPPORTED). */
+LQ_API int lq_encode(const float* w, int rows, int in, const float* M, int d, int D,
+                     uint32_t* packed, int K, float* err, void* stream);
+
 /* Activation lift u = blockdiag(M^T) . T^{-1} . a  (the small matmul T* a
  * computed once before the 1-bit matmul, "Key designs" 4; T on the activation
  * side, "Key designs" 3).

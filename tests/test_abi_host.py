@@ -100,6 +100,14 @@ def _c(v):
                                                      10, 24, _c(P), 0, 49152, None]),
     ("kron plan too big (odd n1)", "lq_lift_activations_kron", [_c(P), 0, 1, 16320, None, _c(P), 255, _c(P), 64,
                                                                 None, _c(P), 10, 24, _c(P), 0, 39168, None]),
+    ("encode d > 16", "lq_encode", [_c(P), 4, 340, _c(P), 17, 24, _c(P), 480, None, None]),
+    ("encode D - d > 24", "lq_encode", [_c(P), 4, 40, _c(P), 4, 29, _c(P), 320, None, None]),
+    ("encode D < d", "lq_encode", [_c(P), 4, 40, _c(P), 8, 4, _c(P), 32, None, None]),
+    ("encode d does not divide in", "lq_encode", [_c(P), 4, 42, _c(P), 4, 12, _c(P), 128, None, None]),
+    ("encode K mismatch", "lq_encode", [_c(P), 4, 40, _c(P), 4, 12, _c(P), 96, None, None]),
+    ("encode null packed", "lq_encode", [_c(P), 4, 40, _c(P), 4, 12, None, 128, None, None]),
+    ("encode misaligned err", "lq_encode", [_c(P), 4, 40, _c(P), 4, 12, _c(P), 128, _c(MIS), None]),
+    ("encode row too long", "lq_encode", [_c(P), 1, 480000, _c(P), 16, 20, _c(P), 600000, None, None]),
 ], ids=lambda c: c[0])
 def test_invalid_arguments_rejected_before_launch(case):
     import bit_lifted_gemm_b200 as lq

@@ -467,3 +467,77 @@ def test_sweep_prefill_b64(lq, D):
     rows = _sample_rows(L.cfg.out, 256, D)
     want = oracle.contract_rows(L.packed, L.s, _oracle_u(L), rows)
     assert rel_err(o[:, rows], want) <= 5e-3
+
+
+# ------------------------------------------------------------------ encoder
+
+def _patterns_from_words(words, rows, nblk, D):
+    """Per-block sign patterns (bit j <=> +1) read back from packed rows: block b
+    of a row occupies bits [b D, (b + 1) D), 32 per word, least significant first."""
+    bits = np.unpackbits(np.ascontiguousarray(words).view(np.uint8).reshape(rows, -1), axis=1, bitorder="little")
+    blk = bits[:, :nblk * D].reshape(rows, nblk, D).astype(np.uint64)
+    return (blk << np.arange(D, dtype=np.uint64)[None, None, :]).sum(axis=2).astype(np.uint64).reshape(-1)
+
+
+def _block_errors(M, wblocks, y, D):
+    s = oracle.patterns_to_signs(y, D).astype(np.float64)
+    return np.sum((wblocks - s @ M.T) ** 2, axis=1)
+
+
+@pytest.mark.parametrize("rows,in_dim,d,D", [
+    (5, 40, 4, 12),    # 256 auxiliary patterns, 8 per lane
+    (3, 640, 10, 24),  # LQ-24/10: 16384 patterns per block
+    (4, 256, 8, 16),   # LQ-16/8
+    (2, 30, 6, 14),    # 70 code bits per row: K = 96 with 26 padding bits
+    (3, 60, 6, 6),     # D = d: no auxiliary coordinates
+    (2, 96, 16, 20),   # d = 16 (the wide variant), 16 patterns: half the lanes idle
+])
+def test_encode_vs_oracle(lq, rows, in_dim, d, D):
+    g = rng_for(62, d * 100 + D, rows)
+    M = g.standard_normal((d, D)) / np.sqrt(D)
+    if D == d:
+        M += 2.0 * np.eye(d)
+    M = M.astype(np.float32)
+    w = g.standard_normal((rows, in_dim)).astype(np.float32)
+    K = oracle.lifted_dim(in_dim, d, D)
+    nblk = in_dim // d
+    packed, err = lq.encode(dev(w), dev(M), K, err=True)
+    words, err = host(packed), host(err)
+    y_gpu = _patterns_from_words(words, rows, nblk, D)
+    Md, wb = oracle.to_f64(M), oracle.to_f64(w).reshape(-1, d)
+    yo, eo = oracle.encode_blocks(Md, wb, nthreads=NTHREADS)
+    # the code is an argmin: identical patterns, or (rarely) a different pattern of equal error
+    same = y_gpu == yo
+    e_gpu = _block_errors(Md, wb, y_gpu, D)
+    assert np.all(same | (np.abs(e_gpu - eo) <= 1e-9 * np.maximum(eo, 1e-300)))
+    assert np.mean(same) >= 0.99
+    assert np.allclose(err.reshape(-1), eo, rtol=1e-6, atol=1e-7)
+    # the words are the library's packing of those patterns (padding bits zero)
+    signs = np.full((rows, K), -1, dtype=np.int8)
+    signs[:, :nblk * D] = oracle.patterns_to_signs(y_gpu, D).reshape(rows, nblk * D)
+    assert np.array_equal(words, oracle.pack_signs(signs))
+
+
+def test_encode_exact_codewords_recovered(lq):
+    """Blocks that are codewords M y* (up to fp32 rounding of w) encode to y*."""
+    g = rng_for(62, 7, 0)
+    d, D, rows, in_dim = 8, 16, 6, 256
+    M = (g.standard_normal((d, D)) / np.sqrt(D)).astype(np.float32)
+    nblk = in_dim // d
+    ystar = g.integers(0, 1 << D, size=rows * nblk, dtype=np.uint64)
+    w = (oracle.patterns_to_signs(ystar, D).astype(np.float64) @ oracle.to_f64(M).T).astype(np.float32)
+    K = oracle.lifted_dim(in_dim, d, D)
+    packed, err = lq.encode(dev(w.reshape(rows, in_dim)), dev(M), K, err=True)
+    assert np.array_equal(_patterns_from_words(host(packed), rows, nblk, D), ystar)
+    assert np.all(host(err) < 1e-9)
+
+
+def test_encode_singular_projection(lq):
+    """A zero row makes M M^T singular: every pattern 0, every error NaN."""
+    d, D, rows, in_dim = 4, 12, 2, 40
+    M = rng_for(62, 8, 0).standard_normal((d, D)).astype(np.float32)
+    M[0, :] = 0.0
+    w = rng_for(62, 9, 0).standard_normal((rows, in_dim)).astype(np.float32)
+    packed, err = lq.encode(dev(w), dev(M), oracle.lifted_dim(in_dim, d, D), err=True)
+    assert np.all(host(packed) == 0)
+    assert np.all(np.isnan(host(err)))
