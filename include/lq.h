@@ -138,7 +138,7 @@ LQ_API int lq_lift_activations_kron(const void* a, int a_dtype, int batch, int i
                                     const float* r2, const float* M, int d, int D,
                                     void* u, int u_dtype, int K, void* stream);
 
-/* Decode 1-bit GEMV, batch 1..16 ("1-bit x float standard GEMM", "Key designs" 4):
+/* Decode 1-bit GEMV, batch 1..16 (the +-1 by float matmul of "Key designs" 4):
  *   o[c][r] = s[r] * sum_k sigma[r][k] * u[c][k],  sigma = +1 if bit set else -1
  *   packed : uint32 [out][K/32]; s : fp32 [out]; u : fp32 [batch][K]
  *   o      : fp32 [batch][out] (written)
