@@ -146,7 +146,6 @@ int lq_encode(const float* w, int rows, int in, const float* M, int d, int D, ui
     if (rows < 1 || in < 1 || d < 1 || d > 16 || D < d || D > 63 || D - d > 24 || in % d != 0)
         return LQ_ERR_INVALID_ARG;
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
-    if (lq::encode_smem(in, d, D) > 200 * 1024) return LQ_ERR_INVALID_ARG;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;

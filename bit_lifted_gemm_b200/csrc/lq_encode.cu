@@ -11,13 +11,14 @@
 // sign(0) = +1; the smallest ||w - M y||^2 wins, the earliest candidate on ties.
 //
 // The search is an offline step whose result is an integer code, so it runs in
-// float64. One CTA per row: it inverts M M^T and M_B once (parallel Gauss-Jordan
-// in shared memory); each warp takes whole blocks. The 32 lanes split the
-// 2^{D-d} patterns and walk their share in Gray-code order, so each step flips
-// one auxiliary coordinate and updates v = w - M_A z, r = M_B^{-1} v and
-// q = M_B y_B incrementally (O(d) per step instead of O(d D)); a warp reduction
-// picks the minimum. The row's patterns are then packed into the 32-per-word
-// layout that lq_gemv reads.
+// float64. Each CTA inverts M M^T and M_B once (parallel Gauss-Jordan in shared
+// memory); the (row, block) units are spread over every warp of the grid. The 32
+// lanes of a warp split the 2^{D-d} patterns of its block and walk their share in
+// Gray-code order, so each step flips one auxiliary coordinate and updates
+// v = w - M_A z, r = M_B^{-1} v and q = M_B y_B incrementally (O(d) per step
+// instead of O(d D)); a warp reduction picks the minimum. The pattern's D bits
+// are ORed into the (zeroed) words of the 32-per-word layout that lq_gemv reads;
+// a block's bits can straddle three words, shared with its neighbours.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -41,13 +42,12 @@ struct EncArgs {
 
 // Shared memory (8-byte units): Md [d][D], P [D][d] = M^T (M M^T)^{-1},
 // Bi [d][d] = M_B^{-1}, G [d][D-d] = M_B^{-1} M_A, gi [d][d] (M M^T, then M_B,
-// as inputs of the inversions), work [d][2d], fac [d], then the row's patterns
-// [nblk] (uint64) and one flag word.
+// as inputs of the inversions), work [d][2d], fac [d] and one flag word.
 struct EncLayout {
-    size_t md, pm, bi, g, gi, wk, fac, pat, flag, total;
+    size_t md, pm, bi, g, gi, wk, fac, flag, total;
 };
 
-__host__ __device__ inline EncLayout enc_layout(int d, int D, int nblk) {
+__host__ __device__ inline EncLayout enc_layout(int d, int D) {
     EncLayout L;
     size_t off = 0;
     auto take = [&off](size_t n8) {
@@ -62,7 +62,6 @@ __host__ __device__ inline EncLayout enc_layout(int d, int D, int nblk) {
     L.gi = take((size_t)d * d);
     L.wk = take((size_t)d * 2 * d);
     L.fac = take((size_t)d);
-    L.pat = take((size_t)nblk);
     L.flag = take(1);
     L.total = off;
     return L;
@@ -258,7 +257,7 @@ template <int MAXD>
 __global__ void __launch_bounds__(EN_THREADS, 1) encode_kernel(const EncArgs p) {
     extern __shared__ __align__(16) uint8_t en_smem[];
     const int d = p.d, D = p.D, na = D - d;
-    const EncLayout L = enc_layout(d, D, p.nblk);
+    const EncLayout L = enc_layout(d, D);
     double* Md = reinterpret_cast<double*>(en_smem + L.md);
     double* P = reinterpret_cast<double*>(en_smem + L.pm);
     double* Bi = reinterpret_cast<double*>(en_smem + L.bi);
@@ -266,7 +265,6 @@ __global__ void __launch_bounds__(EN_THREADS, 1) encode_kernel(const EncArgs p) 
     double* gi = reinterpret_cast<double*>(en_smem + L.gi);
     double* wk = reinterpret_cast<double*>(en_smem + L.wk);
     double* fac = reinterpret_cast<double*>(en_smem + L.fac);
-    uint64_t* pat = reinterpret_cast<uint64_t*>(en_smem + L.pat);
     int* flag = reinterpret_cast<int*>(en_smem + L.flag);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -309,36 +307,49 @@ __global__ void __launch_bounds__(EN_THREADS, 1) encode_kernel(const EncArgs p) 
     const bool singular = *flag != 0;
 
     const int nq = p.K / 32;
-    for (int row = blockIdx.x; row < p.rows; row += gridDim.x) {
-        const float* wrow = p.w + (long long)row * p.in;
-        for (int b = warp; b < p.nblk; b += EN_WARPS) {
-            uint64_t y = 0;
-            double e = __longlong_as_double(0x7ff8000000000000ll);  // NaN: singular M M^T or M_B
-            if (!singular) encode_block<MAXD>(Md, P, Bi, G, d, D, wrow + (long long)b * d, lane, y, e);
-            if (lane == 0) {
-                pat[b] = y;
-                if (p.err) p.err[(long long)row * p.nblk + b] = (float)e;
-            }
+    const long long units = (long long)p.rows * p.nblk;
+    for (long long u = (long long)blockIdx.x * EN_WARPS + warp; u < units; u += (long long)gridDim.x * EN_WARPS) {
+        const int row = (int)(u / p.nblk), b = (int)(u - (long long)row * p.nblk);
+        uint64_t y = 0;
+        double e = __longlong_as_double(0x7ff8000000000000ll);  // NaN: singular M M^T or M_B
+        if (!singular) encode_block<MAXD>(Md, P, Bi, G, d, D, p.w + (long long)row * p.in + (long long)b * d, lane, y, e);
+        if (lane == 0) {
+            if (p.err) p.err[u] = (float)e;
+            // bits [b D, b D + D) of the row: words q, q + 1 and (past 64 bits) q + 2
+            uint32_t* words = p.packed + (long long)row * nq;
+            const long long bit0 = (long long)b * D;
+            const int q = (int)(bit0 >> 5), o = (int)(bit0 & 31);
+            const uint64_t sh = y << o;
+            const uint32_t w0 = (uint32_t)sh, w1 = (uint32_t)(sh >> 32), w2 = o ? (uint32_t)(y >> (64 - o)) : 0u;
+            if (w0) atomicOr(words + q, w0);
+            if (w1) atomicOr(words + q + 1, w1);
+            if (w2) atomicOr(words + q + 2, w2);
         }
-        __syncthreads();
-        // pack: bit k of the row is bit k % D of block k / D; bits past nblk * D are 0
-        for (int q = tid; q < nq; q += EN_THREADS) {
-            uint32_t word = 0;
-            for (int bit = 0; bit < 32; ++bit) {
-                const int k = q * 32 + bit;
-                if (k >= p.nblk * D) break;
-                const int b = k / D;
-                word |= (uint32_t)((pat[b] >> (k - b * D)) & 1ull) << bit;
-            }
-            p.packed[(long long)row * nq + q] = word;
-        }
-        __syncthreads();
     }
 }
 
 }  // namespace
 
-size_t encode_smem(int in, int d, int D) { return enc_layout(d, D, in / d).total; }
+size_t encode_smem(int d, int D) { return enc_layout(d, D).total; }
+
+template <int MAXD>
+cudaError_t launch_encode_t(const EncArgs& p, size_t smem, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(encode_kernel<MAXD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148, per_sm = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_kernel<MAXD>, EN_THREADS, smem) != cudaSuccess ||
+        per_sm < 1) {
+        cudaGetLastError();
+        per_sm = 1;
+    }
+    const long long units = (long long)p.rows * p.nblk;
+    const long long need = (units + EN_WARPS - 1) / EN_WARPS;
+    const int grid = (int)std::max(1ll, std::min(need, (long long)sms * per_sm));
+    encode_kernel<MAXD><<<grid, EN_THREADS, smem, st>>>(p);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_encode(const float* w, int rows, int in, const float* M, int d, int D, uint32_t* packed, int K,
                           float* err, cudaStream_t st) {
@@ -353,21 +364,14 @@ cudaError_t launch_encode(const float* w, int rows, int in, const float* M, int 
     p.D = D;
     p.K = K;
     p.nblk = in / d;
-    const size_t smem = enc_layout(d, D, p.nblk).total;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int grid = std::max(1, std::min(rows, 2 * sms));
-    if (d <= 8) {
-        cudaError_t e = cudaFuncSetAttribute(encode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        encode_kernel<8><<<grid, EN_THREADS, smem, st>>>(p);
-    } else {
-        cudaError_t e = cudaFuncSetAttribute(encode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        encode_kernel<16><<<grid, EN_THREADS, smem, st>>>(p);
-    }
-    return cudaGetLastError();
+    const size_t smem = enc_layout(d, D).total;
+    // the kernel ORs each block's bits into its words
+    cudaError_t e = cudaMemsetAsync(packed, 0, (size_t)rows * (K / 32) * sizeof(uint32_t), st);
+    if (e != cudaSuccess) return e;
+    if (d <= 8) return launch_encode_t<8>(p, smem, st);
+    if (d <= 10) return launch_encode_t<10>(p, smem, st);
+    if (d <= 12) return launch_encode_t<12>(p, smem, st);
+    return launch_encode_t<16>(p, smem, st);
 }
 
 }  // namespace lq

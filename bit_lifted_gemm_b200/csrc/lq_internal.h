@@ -38,7 +38,7 @@ cudaError_t launch_lift_kron(const void* a, bool a_bf16, int batch, int in, cons
 // Encoder (offline): nearest lifted codewords of weight blocks by the
 // pseudo-inverse start plus the 2^{D-d} auxiliary-vector search, float64,
 // written as packed signs. encode_smem gives its shared-memory need.
-size_t encode_smem(int in, int d, int D);
+size_t encode_smem(int d, int D);
 cudaError_t launch_encode(const float* w, int rows, int in, const float* M, int d, int D, uint32_t* packed, int K,
                           float* err, cudaStream_t st);
 

@@ -320,6 +320,18 @@ def test_lift_kron(lq, in_dim, n1, d, D, batch, a_dtype, u_dtype, with_r):
     assert np.all(u[:, k0:] == 0.0)
 
 
+def test_lift_kron_persistent_groups(lq):
+    """1200 tokens in groups of 4: more groups than resident CTAs, so each
+    persistent CTA loops over several groups with its factors kept."""
+    in_dim, n1, d, D, batch = 640, 8, 10, 24, 1200
+    K = oracle.lifted_dim(in_dim, d, D)
+    a, M, kf = _kron_case(in_dim, n1, d, D, batch, "f32", 3)
+    u = host(lq.lift_activations_kron(dev(a), dev(kf.q1), dev(kf.q2), dev(M), K, r1=dev(kf.r1), r2=dev(kf.r2)))
+    want = _kron_oracle_u(a, "f32", M, kf, d, K)
+    assert rel_err(u, want) <= 1e-6
+    assert np.max(np.abs(u - want)) <= 1e-5 * np.max(np.abs(want))
+
+
 def test_lift_kron_then_gemv_vs_oracle(lq):
     """LQ-24/10 decode step with the Kronecker whitening: lift, then the GEMV."""
     L = make_layer(CONFIGS["decode_lq24_10"], 1)
@@ -541,3 +553,18 @@ def test_encode_singular_projection(lq):
     packed, err = lq.encode(dev(w), dev(M), oracle.lifted_dim(in_dim, d, D), err=True)
     assert np.all(host(packed) == 0)
     assert np.all(np.isnan(host(err)))
+
+
+def test_encode_many_rows(lq):
+    """More rows than CTAs (the grid strides over rows), on a cheap shape."""
+    g = rng_for(62, 10, 0)
+    d, D, rows, in_dim = 4, 8, 700, 16
+    M = (g.standard_normal((d, D)) / np.sqrt(D)).astype(np.float32)
+    w = g.standard_normal((rows, in_dim)).astype(np.float32)
+    K = oracle.lifted_dim(in_dim, d, D)
+    words = host(lq.encode(dev(w), dev(M), K))
+    y_gpu = _patterns_from_words(words, rows, in_dim // d, D)
+    yo, eo = oracle.encode_blocks(oracle.to_f64(M), oracle.to_f64(w).reshape(-1, d), nthreads=NTHREADS)
+    e_gpu = _block_errors(oracle.to_f64(M), oracle.to_f64(w).reshape(-1, d), y_gpu, D)
+    assert np.all((y_gpu == yo) | (np.abs(e_gpu - eo) <= 1e-9 * np.maximum(eo, 1e-300)))
+    assert np.mean(y_gpu == yo) >= 0.99
