@@ -28,7 +28,7 @@ cudaError_t launch_lift_tc(const uint16_t* a, int batch, int in, const float* ti
                            void* u, bool u_bf16, int K, unsigned* status, cudaStream_t st);
 
 // Lift with a Kronecker-factored whitening T^{-1} = diag(r2) (Q1 kron Q2) diag(r1)
-// (one thread-block cluster per token group, distributed shared memory).
+// as (Q1 X) Q2^T, each CTA owning a slice of rows of the result.
 // lift_kron_supported tells whether the shapes fit its shared-memory plan.
 bool lift_kron_supported(int batch, int in, int n1, int n2, int d, int D);
 cudaError_t launch_lift_kron(const void* a, bool a_bf16, int batch, int in, const float* r1, const float* q1,

@@ -8,19 +8,18 @@
 // (row-major: element i1 * n2 + i2), (Q1 kron Q2) x is Q1 X Q2^T: in * (n1 + n2)
 // multiply-adds instead of in^2, and (n1^2 + n2^2) floats of factors.
 //
-// One thread-block cluster of C CTAs covers NT tokens; CTA c owns rows
-// [c R, (c + 1) R) of X (R = n1 / C) for all NT tokens:
-//   1. Z = (r1 o X) Q2^T on its rows (rows are independent), kept transposed;
-//   2. cluster barrier, then every CTA gathers all of Z^T from the cluster's
-//      shared memory (distributed shared memory loads);
-//   3. Y = Q1[own rows] Z;
-//   4. a' = r2 o Y and the lift of the d-blocks inside its rows (C is chosen
-//      so that R * n2 is a multiple of d: no block straddles two CTAs).
-// A last cluster barrier keeps each CTA's Z alive until every peer has read it.
-// Both products read their operands along the contraction index in float4:
-// Q1, Q2 and the activations in their natural row-major layout, Z transposed.
-// All arithmetic is fp32 (fp32 accumulation of n2 and then n1 products).
-#include <cooperative_groups.h>
+// The product is taken as Y = (Q1 X) Q2^T. A CTA that owns rows [c R, (c+1) R)
+// of the result needs only its R rows of Q1 and the whole X of its token -- which
+// it reads from global memory -- so a token can be spread over C CTAs with no
+// exchange between them:
+//   1. W = Q1[own rows] (r1 o X)      (R x n2, contraction over n1)
+//   2. Y = W Q2^T                     (R x n2, contraction over n2)
+//   3. a' = r2 o Y and the lift of the d-blocks inside its rows (C is chosen so
+//      that R * n2 is a multiple of d: no block straddles two CTAs).
+// Decode batches (<= 32 tokens) use up to 16 CTAs per token; larger batches keep
+// whole tokens in one CTA, NT per CTA, in persistent CTAs that keep the factors
+// in shared memory across token groups. All arithmetic is fp32 (fp32
+// accumulation of n1 and then n2 products).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -32,10 +31,9 @@
 namespace lq {
 namespace {
 
-namespace cg = cooperative_groups;
-
 constexpr int KR_THREADS = 512;
 constexpr size_t KR_SMEM_BUDGET = 200 * 1024;
+constexpr int KR_BATCH = 4;  // loads issued before their stores in the copy loops
 
 struct KronArgs {
     const void* a;
@@ -47,21 +45,18 @@ struct KronArgs {
     void* u;
     int a_bf16, u_bf16;
     int batch, in, n1, n2, d, D, K;
-    int C, R, Rp, NT;            // CTAs per cluster, rows per CTA (Rp: padded), tokens per cluster
-    int n1p, n2p, ldq, ldz, lda2;  // padded widths and shared-memory row strides (floats)
+    int C, R, Rp, NT;  // CTAs per token group, rows per CTA (Rp: padded to even), tokens per group
+    int n2p, ldq;      // n2 rounded up to 4; row stride of Q2 in shared memory (floats, ldq / 4 odd)
 };
 
 // Shared-memory carve-up (byte offsets, 16-byte aligned), strides in floats:
-//   q2s [n2][ldq]         Q2 rows, zero columns n2 .. n2p
-//   q1s [Rp][n1p]         this CTA's rows of Q1, zero padding
-//   xy  [NT][Rp][n2p]     r1 o X (zero padding), later Y
-//   zt  [NT][n2][ldz]     Z^T of this CTA's rows: zt[t][i2][r] (read by the whole cluster)
-//   za  [NT][n2][lda2]    Z^T of all rows: za[t][i2][j1], zero columns n1 .. n1p
-//   ms  [d][D]            M
-// ldq / 4 and lda2 / 4 are odd: consecutive threads reading consecutive rows
-// in float4 hit distinct banks.
+//   q2s [n2][ldq]        Q2 rows, zero columns n2 .. n2p
+//   q1s [Rp][n1]         this CTA's rows of Q1 (zero padding rows)
+//   xs  [NT][n1][n2p]    r1 o X of the group's tokens, later the compact Y [NT][R * n2]
+//   ws  [NT][Rp][n2p]    W = Q1[own rows] X, zero columns n2 .. n2p
+//   ms  [d][D]           M
 struct KronLayout {
-    size_t q2s, q1s, xy, zt, za, ms, total;
+    size_t q2s, q1s, xs, ws, ms, total;
 };
 
 __host__ __device__ inline KronLayout kron_layout(const KronArgs& p) {
@@ -73,24 +68,62 @@ __host__ __device__ inline KronLayout kron_layout(const KronArgs& p) {
         return o;
     };
     L.q2s = take((size_t)p.n2 * p.ldq * 4);
-    L.q1s = take((size_t)p.Rp * p.n1p * 4);
-    L.xy = take((size_t)p.NT * p.Rp * p.n2p * 4);
-    L.zt = take((size_t)p.NT * p.n2 * p.ldz * 4);
-    L.za = take((size_t)p.NT * p.n2 * p.lda2 * 4);
+    L.q1s = take((size_t)p.Rp * p.n1 * 4);
+    L.xs = take((size_t)p.NT * p.n1 * p.n2p * 4);
+    L.ws = take((size_t)p.NT * p.Rp * p.n2p * 4);
     L.ms = take((size_t)p.d * p.D * 4);
     L.total = off;
     return L;
 }
 
-// C_t[m][n] = sum_{k < Kp} A_t[m][k] * B_t[n][k] for t < nb, m < Mp, n < N, with
-// A_t = A + t * astr, B_t = B + t * bstr (rows at stride lda / ldb; Kp, lda, ldb
-// multiples of 4; Mp a multiple of TM). Work units of one warp: TM rows x 32
-// consecutive columns, one column per lane, so lanes read consecutive B rows
-// (conflict-free with ldb / 4 odd) and share the A rows (broadcast reads).
-// store(t, m, n, value) receives each result.
+// C_t[m][n] = sum_{k < K} A[m][k] * B_t[k][n] (t < nb, m < Mp, n < N): A rows at
+// stride lda, B_t = B + t * bstr rows at stride ldb. A warp's work unit is TM rows
+// x 32 consecutive columns, one column per lane: B reads are consecutive words
+// (conflict-free), A reads are warp-wide broadcasts.
 template <int TM, class Store>
-__device__ __forceinline__ void smem_gemm_abt(const float* A, int lda, size_t astr, const float* B, int ldb,
-                                              size_t bstr, int nb, int Mp, int N, int Kp, Store store) {
+__device__ __forceinline__ void smem_gemm_ab(const float* A, int lda, const float* B, int ldb, size_t bstr, int nb,
+                                             int Mp, int N, int K, Store store) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nblk = (N + 31) >> 5, mg = Mp / TM;
+    const int per_t = mg * nblk;
+    for (int unit = warp; unit < nb * per_t; unit += KR_THREADS / 32) {
+        const int t = unit / per_t, rem = unit - t * per_t;
+        const int g = rem / nblk, n = (rem - g * nblk) * 32 + lane;
+        const bool live = n < N;
+        const float* a = A + (size_t)g * TM * lda;
+        const float* b = B + (size_t)t * bstr + (live ? n : 0);
+        float acc0[TM], acc1[TM];
+#pragma unroll
+        for (int i = 0; i < TM; ++i) acc0[i] = acc1[i] = 0.f;
+        int k = 0;
+#pragma unroll 2
+        for (; k + 1 < K; k += 2) {
+            const float b0 = b[(size_t)k * ldb], b1 = b[(size_t)(k + 1) * ldb];
+#pragma unroll
+            for (int i = 0; i < TM; ++i) {
+                acc0[i] = fmaf(a[(size_t)i * lda + k], b0, acc0[i]);
+                acc1[i] = fmaf(a[(size_t)i * lda + k + 1], b1, acc1[i]);
+            }
+        }
+        if (k < K) {
+            const float b0 = b[(size_t)k * ldb];
+#pragma unroll
+            for (int i = 0; i < TM; ++i) acc0[i] = fmaf(a[(size_t)i * lda + k], b0, acc0[i]);
+        }
+        if (live) {
+#pragma unroll
+            for (int i = 0; i < TM; ++i) store(t, g * TM + i, n, acc0[i] + acc1[i]);
+        }
+    }
+}
+
+// C_t[m][n] = sum_{k < Kp} A_t[m][k] * B[n][k] (t < nb, m < Mp, n < N): A_t = A +
+// t * astr rows at stride lda, B rows at stride ldb (Kp, lda, ldb multiples of 4;
+// ldb / 4 odd). Units of TM rows x 32 consecutive columns; lanes read consecutive
+// B rows in float4 (conflict-free) and share the A rows (broadcast).
+template <int TM, class Store>
+__device__ __forceinline__ void smem_gemm_abt(const float* A, int lda, size_t astr, const float* B, int ldb, int nb,
+                                              int Mp, int N, int Kp, Store store) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nblk = (N + 31) >> 5, mg = Mp / TM;
     const int per_t = mg * nblk;
@@ -99,7 +132,7 @@ __device__ __forceinline__ void smem_gemm_abt(const float* A, int lda, size_t as
         const int g = rem / nblk, n = (rem - g * nblk) * 32 + lane;
         const bool live = n < N;
         const float* a = A + (size_t)t * astr + (size_t)g * TM * lda;
-        const float* b = B + (size_t)t * bstr + (size_t)(live ? n : 0) * ldb;
+        const float* b = B + (size_t)(live ? n : 0) * ldb;
         float acc0[TM], acc1[TM];
 #pragma unroll
         for (int i = 0; i < TM; ++i) acc0[i] = acc1[i] = 0.f;
@@ -122,32 +155,19 @@ __device__ __forceinline__ void smem_gemm_abt(const float* A, int lda, size_t as
     }
 }
 
-template <class Store>
-__device__ __forceinline__ void gemm_abt(const float* A, int lda, size_t astr, const float* B, int ldb, size_t bstr,
-                                         int nb, int Mp, int N, int Kp, Store store) {
-    if (Mp % 4 == 0)
-        smem_gemm_abt<4>(A, lda, astr, B, ldb, bstr, nb, Mp, N, Kp, store);
-    else
-        smem_gemm_abt<2>(A, lda, astr, B, ldb, bstr, nb, Mp, N, Kp, store);
-}
-
-constexpr int KR_BATCH = 4;  // loads issued before their stores in the copy loops
-
 __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs p) {
     // the next kernel on the stream may be scheduled early; it reads u only
     // after its own griddepcontrol.wait, which waits for this grid to complete
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ __align__(16) uint8_t kr_smem[];
-    cg::cluster_group cl = cg::this_cluster();
-    const int c = (int)cl.block_rank();
-    const int row0 = c * p.R;  // first row of X owned by this CTA
+    const int c = (int)(blockIdx.x % p.C);  // row slice of the token group
+    const int row0 = c * p.R;
     const int tid = threadIdx.x;
     const KronLayout L = kron_layout(p);
     float* q2s = reinterpret_cast<float*>(kr_smem + L.q2s);
     float* q1s = reinterpret_cast<float*>(kr_smem + L.q1s);
-    float* xy = reinterpret_cast<float*>(kr_smem + L.xy);
-    float* zt = reinterpret_cast<float*>(kr_smem + L.zt);
-    float* za = reinterpret_cast<float*>(kr_smem + L.za);
+    float* xs = reinterpret_cast<float*>(kr_smem + L.xs);
+    float* ws = reinterpret_cast<float*>(kr_smem + L.ws);
     float* ms = reinterpret_cast<float*>(kr_smem + L.ms);
     // row-by-quad copies: thread (tr, tx) takes quad tx of rows tr, tr + rstep, ...
     const bool vec = (p.n2 & 3) == 0;
@@ -155,7 +175,7 @@ __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs
     const int tr = tid / nq, tx = tid - tr * nq, rstep = KR_THREADS / nq;
 
     // factors first: they do not depend on the kernel before this one, and stay
-    // in shared memory for every token group this cluster takes
+    // in shared memory for every token group this CTA takes
     if (vec && tr < rstep) {
         for (int r0 = tr; r0 < p.n2; r0 += KR_BATCH * rstep) {
             float4 v[KR_BATCH];
@@ -176,16 +196,16 @@ __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs
             q2s[(size_t)i2 * p.ldq + j2] = j2 < p.n2 ? __ldg(p.q2 + (size_t)i2 * p.n2 + j2) : 0.f;
         }
     }
-    for (int idx = tid; idx < p.Rp * p.n1p; idx += KR_THREADS) {
-        const int r = idx / p.n1p, j1 = idx - r * p.n1p;
-        q1s[idx] = r < p.R && j1 < p.n1 ? __ldg(p.q1 + (size_t)(row0 + r) * p.n1 + j1) : 0.f;
+    for (int idx = tid; idx < p.Rp * p.n1; idx += KR_THREADS) {
+        const int r = idx / p.n1, j1 = idx - r * p.n1;
+        q1s[idx] = r < p.R ? __ldg(p.q1 + (size_t)(row0 + r) * p.n1 + j1) : 0.f;
     }
     for (int idx = tid; idx < p.d * p.D; idx += KR_THREADS) ms[idx] = __ldg(p.M + idx);
-    if (p.n1p > p.n1) {  // contraction padding of the gathered Z^T: never overwritten
-        const int pad = p.n1p - p.n1;
-        for (int idx = tid; idx < p.NT * p.n2 * pad; idx += KR_THREADS) {
+    if (p.n2p > p.n2) {  // contraction padding of W: never overwritten
+        const int pad = p.n2p - p.n2;
+        for (int idx = tid; idx < p.NT * p.Rp * pad; idx += KR_THREADS) {
             const int row = idx / pad;
-            za[(size_t)row * p.lda2 + p.n1 + (idx - row * pad)] = 0.f;
+            ws[(size_t)row * p.n2p + p.n2 + (idx - row * pad)] = 0.f;
         }
     }
 
@@ -193,29 +213,30 @@ __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     const int ngroups = (p.batch + p.NT - 1) / p.NT;
-    const int nclusters = (int)(gridDim.x / p.C);
+    const int gstride = (int)(gridDim.x / p.C);
     const int nblk = p.R * p.n2 / p.d;  // d-blocks in this CTA's rows
     const int blk0 = row0 * p.n2 / p.d;
-    const int ycs = p.R * p.n2;         // compact Y of one token: yc[t][r * n2 + i2]
+    const int ycs = p.R * p.n2;         // compact Y of one token: y[t][r * n2 + i2], kept in xs
     const int nbs = KR_THREADS / p.D;   // lift: thread (ljb, lj) takes column lj of blocks ljb, ljb + nbs, ...
     const int lj = tid % p.D, ljb = tid / p.D;
-    for (int grp = (int)(blockIdx.x / p.C); grp < ngroups; grp += nclusters) {
+    const bool tm4 = (p.Rp & 3) == 0;
+    for (int grp = (int)(blockIdx.x / p.C); grp < ngroups; grp += gstride) {
         const int tok0 = grp * p.NT;
 
-        // r1 o X for this CTA's rows of the group's tokens (zero padding)
+        // r1 o X: all n1 rows of the group's tokens (zero rows for missing tokens)
         if (vec) {
             if (tr < rstep) {
                 for (int t = 0; t < p.NT; ++t) {
                     const int tok = tok0 + t;
-                    float* xt = xy + (size_t)t * p.Rp * p.n2p;
-                    for (int r0 = tr; r0 < p.Rp; r0 += KR_BATCH * rstep) {
+                    float* xt = xs + (size_t)t * p.n1 * p.n2p;
+                    for (int r0 = tr; r0 < p.n1; r0 += KR_BATCH * rstep) {
                         float4 v[KR_BATCH];
 #pragma unroll
                         for (int k = 0; k < KR_BATCH; ++k) {
                             const int r = r0 + k * rstep;
                             v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-                            if (r < p.R && tok < p.batch) {
-                                const long long e = (long long)(row0 + r) * p.n2 + 4 * tx;
+                            if (r < p.n1 && tok < p.batch) {
+                                const long long e = (long long)r * p.n2 + 4 * tx;
                                 v[k] = load_act4(p.a, p.a_bf16, (long long)tok * p.in + e);
                                 if (p.r1) {
                                     const float4 w = __ldg(reinterpret_cast<const float4*>(p.r1 + e));
@@ -229,71 +250,50 @@ __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs
 #pragma unroll
                         for (int k = 0; k < KR_BATCH; ++k) {
                             const int r = r0 + k * rstep;
-                            if (r < p.Rp) *reinterpret_cast<float4*>(xt + (size_t)r * p.n2p + 4 * tx) = v[k];
+                            if (r < p.n1) *reinterpret_cast<float4*>(xt + (size_t)r * p.n2p + 4 * tx) = v[k];
                         }
                     }
                 }
             }
         } else {
-            for (int idx = tid; idx < p.NT * p.Rp * p.n2p; idx += KR_THREADS) {
-                const int j2 = idx % p.n2p, row = idx / p.n2p;
-                const int r = row % p.Rp, tok = tok0 + row / p.Rp;
+            for (int idx = tid; idx < p.NT * p.n1 * p.n2p; idx += KR_THREADS) {
+                const int j2 = idx % p.n2p, row = idx / p.n2p;  // row = t * n1 + r
+                const int tok = tok0 + row / p.n1, r = row % p.n1;
                 float v = 0.f;
-                if (r < p.R && j2 < p.n2 && tok < p.batch) {
-                    const long long e = (long long)(row0 + r) * p.n2 + j2;
+                if (j2 < p.n2 && tok < p.batch) {
+                    const long long e = (long long)r * p.n2 + j2;
                     v = load_act(p.a, p.a_bf16, (long long)tok * p.in + e);
                     if (p.r1) v *= __ldg(p.r1 + e);
                 }
-                xy[idx] = v;
+                xs[idx] = v;
             }
         }
         __syncthreads();
 
-        // 1. Z_t = (r1 o X_t) Q2^T on this CTA's rows, stored transposed: zt[t][i2][r]
-        gemm_abt(xy, p.n2p, (size_t)p.Rp * p.n2p, q2s, p.ldq, 0, p.NT, p.Rp, p.n2, p.n2p,
-                 [&](int t, int m, int n, float v) { zt[((size_t)t * p.n2 + n) * p.ldz + m] = v; });
-        cl.sync();  // every CTA's rows of Z are complete and visible to the cluster
-
-        // 2. gather Z^T of all n1 rows: columns [peer R, (peer + 1) R) live in CTA peer
-        if ((p.R & 3) == 0) {
-            const int rq = p.R >> 2, gr = tid / rq, gx = tid - gr * rq, gstep = KR_THREADS / rq;
-            if (gr < gstep) {
-                for (int row = gr; row < p.NT * p.n2; row += gstep) {  // row = t * n2 + i2
-                    float4 v[8];
-#pragma unroll
-                    for (int peer = 0; peer < 8; ++peer)
-                        if (peer < p.C)
-                            v[peer] = *reinterpret_cast<const float4*>(cl.map_shared_rank(zt, peer) +
-                                                                       (size_t)row * p.ldz + 4 * gx);
-#pragma unroll
-                    for (int peer = 0; peer < 8; ++peer)
-                        if (peer < p.C)
-                            *reinterpret_cast<float4*>(za + (size_t)row * p.lda2 + peer * p.R + 4 * gx) = v[peer];
-                }
-            }
-        } else {
-            const int per_peer = p.NT * p.n2 * p.R;
-            for (int q = tid; q < p.C * per_peer; q += KR_THREADS) {
-                const int peer = q / per_peer, rem = q - peer * per_peer;
-                const int x = rem % p.R, row = rem / p.R;
-                za[(size_t)row * p.lda2 + peer * p.R + x] = cl.map_shared_rank(zt, peer)[(size_t)row * p.ldz + x];
-            }
-        }
+        // 1. W_t = Q1[own rows] X_t
+        auto store_w = [&](int t, int m, int n, float v) { ws[((size_t)t * p.Rp + m) * p.n2p + n] = v; };
+        if (tm4)
+            smem_gemm_ab<4>(q1s, p.n1, xs, p.n2p, (size_t)p.n1 * p.n2p, p.NT, p.Rp, p.n2, p.n1, store_w);
+        else
+            smem_gemm_ab<2>(q1s, p.n1, xs, p.n2p, (size_t)p.n1 * p.n2p, p.NT, p.Rp, p.n2, p.n1, store_w);
         __syncthreads();
 
-        // 3. Y_t = Q1[own rows] Z_t, compact into xy (X is no longer needed)
-        gemm_abt(q1s, p.n1p, 0, za, p.lda2, (size_t)p.n2 * p.lda2, p.NT, p.Rp, p.n2, p.n1p,
-                 [&](int t, int m, int n, float v) {
-                     if (m < p.R) xy[(size_t)t * ycs + (size_t)m * p.n2 + n] = v;
-                 });
+        // 2. Y_t = W_t Q2^T, compact into xs (X is no longer needed)
+        auto store_y = [&](int t, int m, int n, float v) {
+            if (m < p.R) xs[(size_t)t * ycs + (size_t)m * p.n2 + n] = v;
+        };
+        if (tm4)
+            smem_gemm_abt<4>(ws, p.n2p, (size_t)p.Rp * p.n2p, q2s, p.ldq, p.NT, p.Rp, p.n2, p.n2p, store_y);
+        else
+            smem_gemm_abt<2>(ws, p.n2p, (size_t)p.Rp * p.n2p, q2s, p.ldq, p.NT, p.Rp, p.n2, p.n2p, store_y);
         __syncthreads();
 
-        // 4. lift the d-blocks of this CTA's rows: u[tok][b D + j] = r2[b] sum_i M[i][j] a'[b d + i]
+        // 3. lift the d-blocks of this CTA's rows: u[tok][b D + j] = r2[b] sum_i M[i][j] a'[b d + i]
         if (ljb < nbs) {
             for (int t = 0; t < p.NT; ++t) {
                 const int tok = tok0 + t;
                 if (tok >= p.batch) break;
-                const float* yt = xy + (size_t)t * ycs;
+                const float* yt = xs + (size_t)t * ycs;
                 for (int b = ljb; b < nblk; b += nbs) {
                     const float* yb = yt + b * p.d;
                     float acc = 0.f;
@@ -312,38 +312,31 @@ __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs
                 if (tok0 + t < p.batch) store_u(p.u, p.u_bf16, (long long)(tok0 + t) * p.K + k, 0.f);
             }
         }
-        // peers have finished reading this CTA's Z^T, and every thread is done
-        // with Y, before the next group overwrites them
-        cl.sync();
+        __syncthreads();  // Y has been read before the next group's X overwrites it
     }
 }
 
-// Decode batches (<= 32 tokens): one token per cluster of C CTAs, C the largest
-// of 8, 4, 2, 1 with n1 % C == 0 and (n1 / C) * n2 a multiple of d, so a token
-// is spread over C SMs. Larger batches: whole tokens per CTA (C = 1), NT of
-// them per CTA (4, 2 or 1, while the shared memory fits), so that no work is
-// split that need not be.
+// Decode batches (<= 32 tokens): C CTAs per token, C the largest of 16, 8, 4, 2,
+// 1 with n1 % C == 0 and (n1 / C) * n2 a multiple of d. Larger batches: whole
+// tokens per CTA (C = 1), NT of them (4, 2 or 1, while the shared memory fits).
 bool kron_plan(int batch, int n1, int n2, int d, int D, KronArgs& p, size_t& smem) {
+    p.n1 = n1;
+    p.n2 = n2;
+    p.d = d;
+    p.D = D;
+    p.n2p = (n2 + 3) & ~3;
+    p.ldq = p.n2p % 8 == 0 ? p.n2p + 4 : p.n2p;
     int C = 1;
     if (batch <= 32)
-        for (int cand = 8; cand >= 1; cand >>= 1)
+        for (int cand = 16; cand >= 1; cand >>= 1)
             if (n1 % cand == 0 && ((n1 / cand) * n2) % d == 0) {
                 C = cand;
                 break;
             }
     if (((n1 / C) * n2) % d != 0) return false;
-    p.n1 = n1;
-    p.n2 = n2;
-    p.d = d;
-    p.D = D;
     p.C = C;
     p.R = n1 / C;
     p.Rp = p.R + (p.R & 1);
-    p.n1p = (n1 + 3) & ~3;
-    p.n2p = (n2 + 3) & ~3;
-    p.ldq = p.n2p % 8 == 0 ? p.n2p + 4 : p.n2p;
-    p.lda2 = p.n1p % 8 == 0 ? p.n1p + 4 : p.n1p;
-    p.ldz = (p.Rp + 3) & ~3;
     for (int NT = batch <= 32 ? 1 : 4;; NT >>= 1) {
         p.NT = NT;
         smem = kron_layout(p).total;
@@ -380,48 +373,29 @@ cudaError_t launch_lift_kron(const void* a, bool a_bf16, int batch, int in, cons
     p.in = in;
     p.K = K;
     static size_t granted[64] = {};
-    int dev = 0;
+    int dev = 0, sms = 148;
     cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (dev >= 64 || granted[dev] < smem) {
         cudaError_t e =
             cudaFuncSetAttribute(lift_kron_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KR_SMEM_BUDGET);
         if (e != cudaSuccess) return e;
         if (dev < 64) granted[dev] = KR_SMEM_BUDGET;
     }
+    // decode: every token group at once; large batches: persistent CTAs, as many
+    // as are resident (512 threads x 128 registers: one per SM)
+    const int ngroups = (batch + p.NT - 1) / p.NT;
+    const int groups_at_once = batch <= 32 ? ngroups : std::max(1, std::min(ngroups, sms / p.C));
     cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(groups_at_once * p.C), 1, 1);
     cfg.blockDim = dim3(KR_THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)p.C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    // persistent clusters: as many as are resident at once (each loops over
-    // token groups with the factors kept in shared memory)
-    static int cached_key[64][3] = {};
-    const int ngroups = (batch + p.NT - 1) / p.NT;
-    int resident = 0;
-    if (dev < 64 && cached_key[dev][0] == p.C && cached_key[dev][1] == (int)smem) {
-        resident = cached_key[dev][2];
-    } else {
-        cfg.gridDim = dim3((unsigned)p.C, 1, 1);
-        if (cudaOccupancyMaxActiveClusters(&resident, lift_kron_kernel, &cfg) != cudaSuccess) {
-            cudaGetLastError();
-            resident = 0;
-        }
-        if (dev < 64 && resident > 0) {
-            cached_key[dev][0] = p.C;
-            cached_key[dev][1] = (int)smem;
-            cached_key[dev][2] = resident;
-        }
-    }
-    if (resident < 1) resident = 1;
-    cfg.gridDim = dim3((unsigned)(std::min(ngroups, resident) * p.C), 1, 1);
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, lift_kron_kernel, p);
 }
 

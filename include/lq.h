@@ -128,7 +128,8 @@ LQ_API int lq_lift_activations(const void* a, int a_dtype, int batch, int in,
  * Kronecker entry ((i1, i2), (j1, j2)) is q1[i1][j1] * q2[i2][j2] with channel
  * i = i1 * n2 + i2, so for one token, X = a reshaped row-major to n1 x n2,
  * (Q1 kron Q2) x = Q1 X Q2^T: in * (n1 + n2) multiply-adds, fp32 throughout.
- * Runs as thread-block clusters (no scratch memory); shapes whose
+ * Computed as (Q1 X) Q2^T with each CTA owning a slice of rows of the result,
+ * so no scratch memory and no exchange between CTAs; shapes whose
  * shared-memory plan does not fit (e.g. a large odd n1) return
  * LQ_ERR_INVALID_ARG. Launched as a programmatic dependent of the preceding
  * kernel; it reads a only after that kernel completes. Requires an sm_100
