@@ -568,3 +568,38 @@ def test_encode_many_rows(lq):
     e_gpu = _block_errors(oracle.to_f64(M), oracle.to_f64(w).reshape(-1, d), y_gpu, D)
     assert np.all((y_gpu == yo) | (np.abs(e_gpu - eo) <= 1e-9 * np.maximum(eo, 1e-300)))
     assert np.mean(y_gpu == yo) >= 0.99
+
+
+# ------------------------------------------------------------------ row-sharded decode
+
+def test_sharded_decode_single_gpu(lq):
+    """ShardedDecode on one GPU: with no process group, and in a 1-rank NCCL group
+    (the all-gather runs), equal to lq_lift_gemv bit for bit."""
+    import datetime
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    from bit_lifted_gemm_b200.sharded import ShardedDecode
+    L = make_layer(CONFIGS["decode_lq20_8"], 4)
+    K = L.cfg.K
+    packed_h = torch.from_numpy(L.packed.view(np.int32))
+    s_h = torch.from_numpy(L.s)
+    a = dev(L.a)
+    _, want = lq.lift_gemv(a, dev(L.M), dev(L.packed), dev(L.s), K, tinv=dev(L.tinv))
+    sd = ShardedDecode(packed_h, s_h, dev(L.M), K, tinv=dev(L.tinv))
+    assert np.array_equal(host(sd(a)), host(want))
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        sd1 = ShardedDecode(packed_h, s_h, dev(L.M), K, tinv=dev(L.tinv))
+        got = sd1(a)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(got), host(want))
+    finally:
+        dist.destroy_process_group()
