@@ -79,8 +79,10 @@ __host__ __device__ inline KronLayout kron_layout(const KronArgs& p) {
 // C_t[m][n] = sum_{k < K} A[m][k] * B_t[k][n] (t < nb, m < Mp, n < N): A rows at
 // stride lda, B_t = B + t * bstr rows at stride ldb. A warp's work unit is TM rows
 // x 32 consecutive columns, one column per lane: B reads are consecutive words
-// (conflict-free), A reads are warp-wide broadcasts.
-template <int TM, class Store>
+// (conflict-free), A reads are warp-wide broadcasts -- four contraction steps per
+// float4 when AV4 (K and lda multiples of 4), which cuts the shared-memory
+// wavefronts per FMA instruction from 5/4 to 12/32 at TM = 8.
+template <int TM, bool AV4, class Store>
 __device__ __forceinline__ void smem_gemm_ab(const float* A, int lda, const float* B, int ldb, size_t bstr, int nb,
                                              int Mp, int N, int K, Store store) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -96,6 +98,20 @@ __device__ __forceinline__ void smem_gemm_ab(const float* A, int lda, const floa
 #pragma unroll
         for (int i = 0; i < TM; ++i) acc0[i] = acc1[i] = 0.f;
         int k = 0;
+        if (AV4) {
+            for (; k < K; k += 4) {
+                const float b0 = b[(size_t)k * ldb], b1 = b[(size_t)(k + 1) * ldb];
+                const float b2 = b[(size_t)(k + 2) * ldb], b3 = b[(size_t)(k + 3) * ldb];
+#pragma unroll
+                for (int i = 0; i < TM; ++i) {
+                    const float4 av = *reinterpret_cast<const float4*>(a + (size_t)i * lda + k);
+                    acc0[i] = fmaf(av.x, b0, acc0[i]);
+                    acc1[i] = fmaf(av.y, b1, acc1[i]);
+                    acc0[i] = fmaf(av.z, b2, acc0[i]);
+                    acc1[i] = fmaf(av.w, b3, acc1[i]);
+                }
+            }
+        }
 #pragma unroll 2
         for (; k + 1 < K; k += 2) {
             const float b0 = b[(size_t)k * ldb], b1 = b[(size_t)(k + 1) * ldb];
@@ -155,6 +171,9 @@ __device__ __forceinline__ void smem_gemm_abt(const float* A, int lda, size_t as
     }
 }
 
+// WIDE: the multi-token (prefill) instantiation with 8-row tiles; the decode
+// instantiation leaves them out and keeps its register count low.
+template <bool WIDE>
 __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs p) {
     // the next kernel on the stream may be scheduled early; it reads u only
     // after its own griddepcontrol.wait, which waits for this grid to complete
@@ -220,6 +239,8 @@ __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs
     const int nbs = KR_THREADS / p.D;   // lift: thread (ljb, lj) takes column lj of blocks ljb, ljb + nbs, ...
     const int lj = tid % p.D, ljb = tid / p.D;
     const bool tm4 = (p.Rp & 3) == 0;
+    // multi-token groups (prefill): 8-row tiles, Q1 read four steps per float4
+    const bool wide = WIDE && (p.Rp & 7) == 0 && (p.n1 & 3) == 0;
     for (int grp = (int)(blockIdx.x / p.C); grp < ngroups; grp += gstride) {
         const int tok0 = grp * p.NT;
 
@@ -272,17 +293,21 @@ __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs
 
         // 1. W_t = Q1[own rows] X_t
         auto store_w = [&](int t, int m, int n, float v) { ws[((size_t)t * p.Rp + m) * p.n2p + n] = v; };
-        if (tm4)
-            smem_gemm_ab<4>(q1s, p.n1, xs, p.n2p, (size_t)p.n1 * p.n2p, p.NT, p.Rp, p.n2, p.n1, store_w);
+        if (wide)
+            smem_gemm_ab<8, true>(q1s, p.n1, xs, p.n2p, (size_t)p.n1 * p.n2p, p.NT, p.Rp, p.n2, p.n1, store_w);
+        else if (tm4)
+            smem_gemm_ab<4, false>(q1s, p.n1, xs, p.n2p, (size_t)p.n1 * p.n2p, p.NT, p.Rp, p.n2, p.n1, store_w);
         else
-            smem_gemm_ab<2>(q1s, p.n1, xs, p.n2p, (size_t)p.n1 * p.n2p, p.NT, p.Rp, p.n2, p.n1, store_w);
+            smem_gemm_ab<2, false>(q1s, p.n1, xs, p.n2p, (size_t)p.n1 * p.n2p, p.NT, p.Rp, p.n2, p.n1, store_w);
         __syncthreads();
 
         // 2. Y_t = W_t Q2^T, compact into xs (X is no longer needed)
         auto store_y = [&](int t, int m, int n, float v) {
             if (m < p.R) xs[(size_t)t * ycs + (size_t)m * p.n2 + n] = v;
         };
-        if (tm4)
+        if (wide)
+            smem_gemm_abt<8>(ws, p.n2p, (size_t)p.Rp * p.n2p, q2s, p.ldq, p.NT, p.Rp, p.n2, p.n2p, store_y);
+        else if (tm4)
             smem_gemm_abt<4>(ws, p.n2p, (size_t)p.Rp * p.n2p, q2s, p.ldq, p.NT, p.Rp, p.n2, p.n2p, store_y);
         else
             smem_gemm_abt<2>(ws, p.n2p, (size_t)p.Rp * p.n2p, q2s, p.ldq, p.NT, p.Rp, p.n2, p.n2p, store_y);
@@ -377,8 +402,11 @@ cudaError_t launch_lift_kron(const void* a, bool a_bf16, int batch, int in, cons
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (dev >= 64 || granted[dev] < smem) {
-        cudaError_t e =
-            cudaFuncSetAttribute(lift_kron_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KR_SMEM_BUDGET);
+        cudaError_t e = cudaFuncSetAttribute(lift_kron_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)KR_SMEM_BUDGET);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(lift_kron_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)KR_SMEM_BUDGET);
         if (e != cudaSuccess) return e;
         if (dev < 64) granted[dev] = KR_SMEM_BUDGET;
     }
@@ -396,7 +424,8 @@ cudaError_t launch_lift_kron(const void* a, bool a_bf16, int batch, int in, cons
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, lift_kron_kernel, p);
+    return p.NT > 1 ? cudaLaunchKernelEx(&cfg, lift_kron_kernel<true>, p)
+                    : cudaLaunchKernelEx(&cfg, lift_kron_kernel<false>, p);
 }
 
 }  // namespace lq

@@ -298,6 +298,7 @@ def _kron_oracle_u(a, a_dtype, M, kf, d, K, with_r=True):
     (5120, 64, 10, 24, 16, "bf16", "f32", True),
     (8192, 64, 8, 20, 2, "bf16", "f32", True),    # LQ-20/8 layer, 64 x 128 factors
     (70, 7, 5, 18, 2, "f32", "f32", True),        # odd n1: one CTA per token; n2 = 10 padded; K tail of 4
+    (70, 7, 5, 18, 40, "f32", "f32", True),       # odd n1, 4 tokens per CTA: the narrow multi-token tiles
     (48, 8, 4, 8, 3, "f32", "f32", True),         # d-blocks straddle rows of X; clusters of 4
     (640, 8, 10, 24, 70, "bf16", "bf16", True),   # 4 tokens per cluster, ragged last cluster, bf16 output
     (5120, 64, 10, 24, 40, "bf16", "bf16", True), # prefill-sized batch on the LQ-24/10 layer
