@@ -24,7 +24,7 @@ LQ_F32, LQ_BF16 = 0, 1
 
 SYMBOLS = ("lq_status_str", "lq_lifted_dim", "lq_pack_signs", "lq_unpack_signs", "lq_lift_activations",
            "lq_lift_activations_kron", "lq_gemv", "lq_lift_gemv", "lq_gemm", "lq_encode",
-           "lq_get_device_status")
+           "lq_selftest_wait_timeout", "lq_get_device_status")
 
 
 class LQError(RuntimeError):
@@ -56,6 +56,8 @@ def _load() -> ctypes.CDLL:
     lib.lq_lift_gemv.argtypes = [p, i, i, i, p, i, p, i, i, p, p, i, i, p, p, p]
     lib.lq_gemm.restype = i
     lib.lq_encode.restype = i
+    lib.lq_selftest_wait_timeout.restype = i
+    lib.lq_selftest_wait_timeout.argtypes = [ctypes.c_uint, p]
     lib.lq_encode.argtypes = [p, i, i, p, i, i, p, i, p, p]
     lib.lq_gemm.argtypes = [p, p, i, i, p, i, p, p]
     lib.lq_get_device_status.restype = i

@@ -152,6 +152,17 @@ int lq_encode(const float* w, int rows, int in, const float* M, int d, int D, ui
     return from_cuda(lq::launch_encode(w, rows, in, M, d, D, packed, K, err, static_cast<cudaStream_t>(stream)));
 }
 
+int lq_selftest_wait_timeout(unsigned limit_us, void* stream) {
+    if (limit_us < 1 || limit_us > 1000000) return LQ_ERR_INVALID_ARG;
+    const int sm = is_sm100();
+    if (sm < 0) return LQ_ERR_CUDA;
+    if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    int err = LQ_OK;
+    unsigned* status = status_word(&err);
+    if (!status) return err;
+    return from_cuda(lq::launch_selftest_wait_timeout(limit_us, status, static_cast<cudaStream_t>(stream)));
+}
+
 int lq_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u, int batch, float* o,
             void* stream) {
     if (!packed || !s || !u || !o) return LQ_ERR_INVALID_ARG;

@@ -42,6 +42,9 @@ size_t encode_smem(int d, int D);
 cudaError_t launch_encode(const float* w, int rows, int in, const float* M, int d, int D, uint32_t* packed, int K,
                           float* err, cudaStream_t st);
 
+// Self-test of the bounded waits: one wait that nothing completes, limit_us long.
+cudaError_t launch_selftest_wait_timeout(unsigned limit_us, unsigned* status, cudaStream_t st);
+
 // Decode GEMV (integer tensor cores; u quantized per CTA). `status` is the
 // device status word that bounded waits report to.
 cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u,

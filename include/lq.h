@@ -185,6 +185,14 @@ LQ_API int lq_lift_gemv(const void* a, int a_dtype, int batch, int in, const flo
 LQ_API int lq_gemm(const uint32_t* packed, const float* s, int out, int K,
             const uint16_t* u_bf16, int tokens, float* o, void* stream);
 
+/* Self-test of the failure reporting: launches one thread that waits, through
+ * the bounded-wait helper the GEMV and GEMM use, on an mbarrier that nothing
+ * ever completes. After limit_us microseconds (1 .. 1000000) the wait gives up,
+ * latches LQ_ERR_TIMEOUT in the device status word and the kernel returns; the
+ * next lq_get_device_status reports it. Nothing faults or hangs. Requires an
+ * sm_100 device (else LQ_ERR_UNSUPPORTED). */
+LQ_API int lq_selftest_wait_timeout(unsigned limit_us, void* stream);
+
 /* Synchronizes `stream`, then returns and clears the device status word of the
  * current device: LQ_OK, or LQ_ERR_TIMEOUT if a kernel gave up a bounded wait
  * since the last call. Returns LQ_ERR_CUDA if the synchronize fails. */

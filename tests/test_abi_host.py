@@ -107,6 +107,8 @@ def _c(v):
     ("encode K mismatch", "lq_encode", [_c(P), 4, 40, _c(P), 4, 12, _c(P), 96, None, None]),
     ("encode null packed", "lq_encode", [_c(P), 4, 40, _c(P), 4, 12, None, 128, None, None]),
     ("encode misaligned err", "lq_encode", [_c(P), 4, 40, _c(P), 4, 12, _c(P), 128, _c(MIS), None]),
+    ("selftest limit 0", "lq_selftest_wait_timeout", [0, None]),
+    ("selftest limit above 1 s", "lq_selftest_wait_timeout", [2000000, None]),
 ], ids=lambda c: c[0])
 def test_invalid_arguments_rejected_before_launch(case):
     import bit_lifted_gemm_b200 as lq

@@ -604,3 +604,19 @@ def test_sharded_decode_single_gpu(lq):
         assert np.array_equal(host(got), host(want))
     finally:
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ failure reporting
+
+def test_bounded_wait_reports_timeout(lq):
+    """A wait that nothing completes gives up after its limit (1 ms here), latches
+    LQ_ERR_TIMEOUT for lq_get_device_status, which then clears it, and leaves the
+    context usable."""
+    assert lq.get_device_status() == lq.LQ_OK
+    assert lq.lib.lq_selftest_wait_timeout(1000, None) == lq.LQ_OK
+    assert lq.get_device_status() == lq.LQ_ERR_TIMEOUT
+    assert lq.get_device_status() == lq.LQ_OK
+    L = make_layer(CONFIGS["tiny"], 2)
+    o = host(lq.gemv(dev(L.packed), dev(L.s), _gpu_u(lq, L)))
+    want = oracle.contract(L.packed, L.s, _oracle_u(L))
+    assert rel_err(o, want) <= 1e-5
