@@ -114,3 +114,15 @@ def test_invalid_arguments_rejected_before_launch(case):
     import bit_lifted_gemm_b200 as lq
     _, fn, args = case
     assert getattr(lq.lib, fn)(*args) == lq.LQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("lang,compiler", [("c", "gcc"), ("c++", "g++")])
+def test_header_compiles_standalone(lang, compiler):
+    """include/lq.h is a plain C header (also usable from C++)."""
+    import shutil
+    import subprocess
+    if shutil.which(compiler) is None:
+        pytest.skip(f"{compiler} not installed")
+    r = subprocess.run([compiler, "-fsyntax-only", "-Wall", "-Wextra", "-Werror", "-x", lang,
+                        os.path.join(ROOT, "include", "lq.h")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
