@@ -620,3 +620,43 @@ def test_bounded_wait_reports_timeout(lq):
     o = host(lq.gemv(dev(L.packed), dev(L.s), _gpu_u(lq, L)))
     want = oracle.contract(L.packed, L.s, _oracle_u(L))
     assert rel_err(o, want) <= 1e-5
+
+
+# ------------------------------------------------------------------ bench-size sampled checks
+
+def test_lift_kron_prefill_bench_size_sampled(lq):
+    """The 2048-token LQ-24/10 prefill lift as bench.py runs it (64 x 80 factors,
+    bf16 activations and u, persistent CTAs with 8-row tiles), checked on sampled
+    tokens that the oracle computes one by one."""
+    from datagen import make_kron_factors
+    cfg = CONFIGS["decode_lq24_10"]
+    kf = make_kron_factors(cfg.in_dim, 64, cfg.d, cfg.index)
+    L = make_layer(CONFIGS["prefill_lq24_10"], 2048, packed=False)
+    u = host(lq.lift_activations_kron(dev(L.a), dev(kf.q1), dev(kf.q2), dev(L.M), cfg.K, r1=dev(kf.r1),
+                                      r2=dev(kf.r2), u_dtype="bf16"))
+    toks = np.unique(np.concatenate([rng_for(63, 1, 0).choice(2048, size=6, replace=False), [0, 2047]]))
+    want = _kron_oracle_u(L.a[toks], "bf16", L.M, kf, cfg.d, cfg.K)
+    got = oracle.to_f64(u[toks], "bf16")
+    assert np.all(np.abs(got - want) <= _bf16_ulp(want) + 1e-6 * np.max(np.abs(want)))
+
+
+def test_encode_bench_size_sampled(lq):
+    """The LQ-24/10 encoder input bench.py times (26 x 5120 seeded weights), checked
+    on sampled blocks that the oracle searches one by one."""
+    d, D, rows, in_dim = 10, 24, 26, 5120
+    g = np.random.default_rng(0x4C51 + D)
+    M = (g.standard_normal((d, D)) / np.sqrt(D)).astype(np.float32)
+    w = g.standard_normal((rows, in_dim)).astype(np.float32)
+    K = oracle.lifted_dim(in_dim, d, D)
+    packed, err = lq.encode(dev(w), dev(M), K, err=True)
+    nblk = in_dim // d
+    y_gpu = _patterns_from_words(host(packed), rows, nblk, D)
+    e_gpu = host(err).reshape(-1)
+    pick = rng_for(63, 2, 0).choice(rows * nblk, size=200, replace=False)
+    wb = oracle.to_f64(w).reshape(-1, d)[pick]
+    yo, eo = oracle.encode_blocks(oracle.to_f64(M), wb, nthreads=NTHREADS)
+    same = y_gpu[pick] == yo
+    e_pick = _block_errors(oracle.to_f64(M), wb, y_gpu[pick], D)
+    assert np.all(same | (np.abs(e_pick - eo) <= 1e-9 * np.maximum(eo, 1e-300)))
+    assert np.mean(same) >= 0.99
+    assert np.allclose(e_gpu[pick], eo, rtol=1e-6, atol=1e-7)
