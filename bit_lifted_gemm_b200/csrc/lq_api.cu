@@ -5,6 +5,8 @@
 // kernels set when they give up.
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "lq.h"
 #include "lq_internal.h"
@@ -18,6 +20,15 @@ constexpr int kMaxDevices = 64;
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? LQ_OK : LQ_ERR_CUDA; }
+
+// Host-side fault injection for the error-path tests (no device fault is ever
+// made): LQ_FAULT=launch makes every compute entry point return LQ_ERR_CUDA after
+// its argument checks, without launching; LQ_FAULT=timeout makes
+// lq_get_device_status report LQ_ERR_TIMEOUT without touching the device.
+bool fault_is(const char* mode) {
+    const char* f = getenv("LQ_FAULT");
+    return f && strcmp(f, mode) == 0;
+}
 
 // True if kernels may load and store through p as given: device or managed
 // memory, or page-locked host memory that unified addressing maps at the same
@@ -93,12 +104,14 @@ int lq_lifted_dim(int in, int d, int D) {
 int lq_pack_signs(const int8_t* signs_pm1, int out, int K, uint32_t* packed, void* stream) {
     if (!signs_pm1 || !packed || !aligned16(signs_pm1) || !aligned16(packed)) return LQ_ERR_INVALID_ARG;
     if (out < 1 || K < 32 || K % 32 != 0) return LQ_ERR_INVALID_ARG;
+    if (fault_is("launch")) return LQ_ERR_CUDA;
     return from_cuda(lq::launch_pack(signs_pm1, out, K, packed, static_cast<cudaStream_t>(stream)));
 }
 
 int lq_unpack_signs(const uint32_t* packed, int out, int K, int8_t* signs_pm1, void* stream) {
     if (!signs_pm1 || !packed || !aligned16(signs_pm1) || !aligned16(packed)) return LQ_ERR_INVALID_ARG;
     if (out < 1 || K < 32 || K % 32 != 0) return LQ_ERR_INVALID_ARG;
+    if (fault_is("launch")) return LQ_ERR_CUDA;
     return from_cuda(lq::launch_unpack(packed, out, K, signs_pm1, static_cast<cudaStream_t>(stream)));
 }
 
@@ -111,6 +124,7 @@ int lq_lift_activations(const void* a, int a_dtype, int batch, int in, const flo
     if (batch < 1 || in < 1 || d < 1 || d > 64 || D < 1 || D > 256 || d * D > 4096) return LQ_ERR_INVALID_ARG;
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
     if (tinv && (tblk < 1 || tblk > 256 || in % tblk != 0)) return LQ_ERR_INVALID_ARG;
+    if (fault_is("launch")) return LQ_ERR_CUDA;
     int err = LQ_OK;
     unsigned* status = status_word(&err);
     if (!status) return err;
@@ -132,6 +146,7 @@ int lq_lift_activations_kron(const void* a, int a_dtype, int batch, int in, cons
     if (n1 < 1 || n1 > 256 || n2 < 1 || n2 > 128 || n1 * n2 != in || in % d != 0) return LQ_ERR_INVALID_ARG;
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
     if (!lq::lift_kron_supported(batch, in, n1, n2, d, D)) return LQ_ERR_INVALID_ARG;
+    if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
@@ -146,6 +161,7 @@ int lq_encode(const float* w, int rows, int in, const float* M, int d, int D, ui
     if (rows < 1 || in < 1 || d < 1 || d > 16 || D < d || D > 63 || D - d > 24 || in % d != 0)
         return LQ_ERR_INVALID_ARG;
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
+    if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
@@ -154,6 +170,7 @@ int lq_encode(const float* w, int rows, int in, const float* M, int d, int D, ui
 
 int lq_selftest_wait_timeout(unsigned limit_us, void* stream) {
     if (limit_us < 1 || limit_us > 1000000) return LQ_ERR_INVALID_ARG;
+    if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
@@ -168,6 +185,7 @@ int lq_gemv(const uint32_t* packed, const float* s, int out, int K, const float*
     if (!packed || !s || !u || !o) return LQ_ERR_INVALID_ARG;
     if (!aligned16(packed) || !aligned16(s) || !aligned16(u) || !aligned16(o)) return LQ_ERR_INVALID_ARG;
     if (out < 1 || K < 32 || K % 32 != 0 || batch < 1 || batch > 16) return LQ_ERR_INVALID_ARG;
+    if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
@@ -189,6 +207,7 @@ int lq_lift_gemv(const void* a, int a_dtype, int batch, int in, const float* tin
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
     if (tinv && (tblk < 1 || tblk > 256 || in % tblk != 0)) return LQ_ERR_INVALID_ARG;
     if (out < 1) return LQ_ERR_INVALID_ARG;
+    if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
@@ -205,6 +224,7 @@ int lq_gemm(const uint32_t* packed, const float* s, int out, int K, const uint16
     if (!packed || !s || !u_bf16 || !o) return LQ_ERR_INVALID_ARG;
     if (!aligned16(packed) || !aligned16(s) || !aligned16(u_bf16) || !aligned16(o)) return LQ_ERR_INVALID_ARG;
     if (out < 1 || K < 32 || K % 32 != 0 || tokens < 1) return LQ_ERR_INVALID_ARG;
+    if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
@@ -215,6 +235,7 @@ int lq_gemm(const uint32_t* packed, const float* s, int out, int K, const uint16
 }
 
 int lq_get_device_status(void* stream) {
+    if (fault_is("timeout")) return LQ_ERR_TIMEOUT;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return LQ_ERR_CUDA;
     unsigned v = 0;
     if (cudaMemcpyFromSymbol(&v, g_lq_status, sizeof(v)) != cudaSuccess) return LQ_ERR_CUDA;

@@ -23,6 +23,11 @@
  *    by lq_get_device_status().
  *  - Packed signs: 32 per uint32, least significant bit first along the
  *    lifted axis, bit 1 = +1, row-major [out][K/32].
+ *  - Fault injection for error-path tests (host side only): with the
+ *    environment variable LQ_FAULT=launch every compute call returns
+ *    LQ_ERR_CUDA after its argument checks, without launching; with
+ *    LQ_FAULT=timeout lq_get_device_status returns LQ_ERR_TIMEOUT without
+ *    touching the device.
  *  - bf16 values are passed as their uint16 bit patterns.
  */
 #ifndef LQ_H

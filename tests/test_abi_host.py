@@ -126,3 +126,23 @@ def test_header_compiles_standalone(lang, compiler):
     r = subprocess.run([compiler, "-fsyntax-only", "-Wall", "-Wextra", "-Werror", "-x", lang,
                         os.path.join(ROOT, "include", "lq.h")], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_fault_injection_timeout(monkeypatch):
+    """LQ_FAULT=timeout: lq_get_device_status reports a timeout without a device."""
+    import bit_lifted_gemm_b200 as lq
+    monkeypatch.setenv("LQ_FAULT", "timeout")
+    assert lq.lib.lq_get_device_status(None) == lq.LQ_ERR_TIMEOUT
+    assert lq.lib.lq_status_str(lq.LQ_ERR_TIMEOUT)
+
+
+def test_fault_injection_launch(monkeypatch):
+    """LQ_FAULT=launch: valid calls return LQ_ERR_CUDA without touching their
+    pointers; argument checks still come first."""
+    import bit_lifted_gemm_b200 as lq
+    monkeypatch.setenv("LQ_FAULT", "launch")
+    assert lq.lib.lq_pack_signs(_c(P), 4, 32, _c(P), None) == lq.LQ_ERR_CUDA
+    assert lq.lib.lq_gemv(_c(P), _c(P), 8, 64, _c(P), 1, _c(P), None) == lq.LQ_ERR_CUDA
+    assert lq.lib.lq_gemm(_c(P), _c(P), 8, 64, _c(P), 4, _c(P), None) == lq.LQ_ERR_CUDA
+    assert lq.lib.lq_encode(_c(P), 4, 40, _c(P), 4, 12, _c(P), 128, None, None) == lq.LQ_ERR_CUDA
+    assert lq.lib.lq_gemv(_c(P), _c(P), 8, 64, _c(P), 0, _c(P), None) == lq.LQ_ERR_INVALID_ARG
