@@ -25,7 +25,8 @@ number (pinned-host activations in, output back to the host, inside the timed
 region: zero-copy, the lift loading and the GEMV storing the host buffers, with
 the copy-engine variant beside it), sampled SM clocks, the float64 oracle timed on the host cores, and
 secondary results (prefill GEMM TFLOP/s, the LQ-20/8 batch sweep, the LQ-D/8
-bit-width sweep).
+bit-width sweep, the Kronecker-whitened lift, the encoder's seconds per
+million weights).
 """
 
 from __future__ import annotations
