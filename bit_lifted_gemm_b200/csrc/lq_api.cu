@@ -185,6 +185,7 @@ int lq_gemv(const uint32_t* packed, const float* s, int out, int K, const float*
     if (!packed || !s || !u || !o) return LQ_ERR_INVALID_ARG;
     if (!aligned16(packed) || !aligned16(s) || !aligned16(u) || !aligned16(o)) return LQ_ERR_INVALID_ARG;
     if (out < 1 || K < 32 || K % 32 != 0 || batch < 1 || batch > 16) return LQ_ERR_INVALID_ARG;
+    if (!lq::gemv_supported(out, K, batch)) return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
@@ -206,7 +207,7 @@ int lq_lift_gemv(const void* a, int a_dtype, int batch, int in, const float* tin
         return LQ_ERR_INVALID_ARG;
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
     if (tinv && (tblk < 1 || tblk > 256 || in % tblk != 0)) return LQ_ERR_INVALID_ARG;
-    if (out < 1) return LQ_ERR_INVALID_ARG;
+    if (out < 1 || !lq::gemv_supported(out, K, batch)) return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;

@@ -688,7 +688,7 @@ Plan make_plan(int out, int kw, int batch) {
             }
         }
     }
-    return pl;  // not reached: one column with enough chunks always fits
+    return pl;  // nothing fits: the CTA's row partials (maxgroups) are too many; gemv_supported says so
 }
 
 template <int TS, int STAGES, bool TMA, bool USTAGE>
@@ -734,6 +734,10 @@ cudaError_t launch_planned(const CUtensorMap& wmap, const CUtensorMap& umap, con
 }
 
 }  // namespace
+
+bool gemv_supported(int out, int K, int batch) {
+    return make_plan(out, K / 32, batch).smem <= kSmemBudget;
+}
 
 cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u, int batch, float* o,
                         unsigned* status, cudaStream_t st) {

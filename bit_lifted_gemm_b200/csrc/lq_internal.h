@@ -47,6 +47,9 @@ cudaError_t launch_selftest_wait_timeout(unsigned limit_us, unsigned* status, cu
 
 // Decode GEMV (integer tensor cores; u quantized per CTA). `status` is the
 // device status word that bounded waits report to.
+// Whether the GEMV's launch plan fits in shared memory for this shape (each CTA
+// keeps 64-bit partial sums for its rows, so very large `out` does not fit).
+bool gemv_supported(int out, int K, int batch);
 cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u,
                         int batch, float* o, unsigned* status, cudaStream_t st);
 

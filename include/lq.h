@@ -152,8 +152,10 @@ LQ_API int lq_lift_activations_kron(const void* a, int a_dtype, int batch, int i
  * u is converted per K-part and column to 24-bit fixed point (error <= 2^-22 of
  * the part's largest |u|); the sign contraction itself is exact integer
  * arithmetic, so the result is within ~1e-6 relative (Frobenius) of the exact
- * value. Deterministic. Needs no scratch memory. Requires an sm_100 device
- * (else LQ_ERR_UNSUPPORTED). */
+ * value. Deterministic. Needs no scratch memory. Each CTA keeps 64-bit partial
+ * sums for its rows in shared memory, which bounds `out` (about 3.1 million rows
+ * for K in the tens of thousands on a 148-SM B200); larger shapes return
+ * LQ_ERR_INVALID_ARG. Requires an sm_100 device (else LQ_ERR_UNSUPPORTED). */
 LQ_API int lq_gemv(const uint32_t* packed, const float* s, int out, int K,
             const float* u, int batch, float* o, void* stream);
 

@@ -146,3 +146,12 @@ def test_fault_injection_launch(monkeypatch):
     assert lq.lib.lq_gemm(_c(P), _c(P), 8, 64, _c(P), 4, _c(P), None) == lq.LQ_ERR_CUDA
     assert lq.lib.lq_encode(_c(P), 4, 40, _c(P), 4, 12, _c(P), 128, None, None) == lq.LQ_ERR_CUDA
     assert lq.lib.lq_gemv(_c(P), _c(P), 8, 64, _c(P), 0, _c(P), None) == lq.LQ_ERR_INVALID_ARG
+
+
+def test_gemv_rejects_rows_beyond_the_plan():
+    """Row counts whose per-CTA partial sums cannot fit in shared memory are
+    refused before any launch (a 2^24-row exhaustive codebook, for instance)."""
+    import bit_lifted_gemm_b200 as lq
+    assert lq.lib.lq_gemv(_c(P), _c(P), 1 << 24, 32, _c(P), 1, _c(P), None) == lq.LQ_ERR_INVALID_ARG
+    assert lq.lib.lq_lift_gemv(_c(P), 0, 1, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 1 << 24, 1536,
+                               _c(P), _c(P), None) == lq.LQ_ERR_INVALID_ARG
