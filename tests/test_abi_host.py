@@ -155,3 +155,17 @@ def test_gemv_rejects_rows_beyond_the_plan():
     assert lq.lib.lq_gemv(_c(P), _c(P), 1 << 24, 32, _c(P), 1, _c(P), None) == lq.LQ_ERR_INVALID_ARG
     assert lq.lib.lq_lift_gemv(_c(P), 0, 1, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 1 << 24, 1536,
                                _c(P), _c(P), None) == lq.LQ_ERR_INVALID_ARG
+
+
+def test_gemv_plan_fits_every_configured_layer():
+    """The shape check accepts every configured decode layer and batch: on a
+    host without a GPU such calls get past argument checking (to LQ_ERR_CUDA or
+    LQ_ERR_UNSUPPORTED), never LQ_ERR_INVALID_ARG."""
+    import bit_lifted_gemm_b200 as lq
+    from datagen import CONFIGS
+    for cfg in CONFIGS.values():
+        if cfg.kind == "prefill":
+            continue
+        for batch in (1, 2, 4, 8, 16):
+            rc = lq.lib.lq_gemv(_c(P), _c(P), cfg.out, cfg.K, _c(P), batch, _c(P), None)
+            assert rc != lq.LQ_ERR_INVALID_ARG, (cfg.name, batch)
