@@ -54,8 +54,8 @@ METRIC = "decode GEMV packed-weight GB/s (% of HBM) and prefill TFLOP/s, per LQ-
 def workload_config(cfg, name, world):
     return {"workload": name, "in": cfg.in_dim, "out": cfg.out, "d": cfg.d, "D": cfg.D, "K": cfg.K,
             "batch": 1, "tblk": cfg.tblk, "step": "lq_lift_gemv (lift + gemv)", "parallelism": f"replicas{world}",
-            "arith": "lift fp32; u as 24-bit fixed point in three int8 digit planes; u8 x s8 -> s32 MMA (exact); "
-                     "fp32 output"}
+            "arith": "lift fp32; u as 32-bit fixed point in four int8 digit planes (quantized once per call); "
+                     "u8 x s8 -> s32 MMA (exact); fp32 output"}
 
 
 # ------------------------------------------------------------------ helpers
@@ -206,6 +206,8 @@ class DecodeLayer:
         self.u = [torch.empty((batch, cfg.K), dtype=torch.float32, device=dev) for _ in range(copies)]
         self.o = [torch.empty((batch, cfg.out), dtype=torch.float32, device=dev) for _ in range(copies)]
         self.o_host = [torch.empty((batch, cfg.out), dtype=torch.float32).pin_memory() for _ in range(copies)]
+        # one workspace serves every step: the steps run in stream order
+        self.ws = lq.gemv_workspace(cfg.out, cfg.K, batch, dev)
         self.copies = copies
         self.lq = lq
 
@@ -213,7 +215,8 @@ class DecodeLayer:
         lq, c = self.lq, self.cfg
         if with_copies:
             self.a[i].copy_(self.a_host[i], non_blocking=True)
-        lq.lift_gemv(self.a[i], self.M, self.packed[i], self.s[i], c.K, tinv=self.tinv[i], u=self.u[i], out=self.o[i])
+        lq.lift_gemv(self.a[i], self.M, self.packed[i], self.s[i], c.K, tinv=self.tinv[i], u=self.u[i], out=self.o[i],
+                     workspace=self.ws)
         if with_copies:
             self.o_host[i].copy_(self.o[i], non_blocking=True)
 
@@ -222,10 +225,10 @@ class DecodeLayer:
         from pinned host memory and the GEMV stores o there."""
         lq, c = self.lq, self.cfg
         lq.lift_gemv(self.a_host[i], self.M, self.packed[i], self.s[i], c.K, tinv=self.tinv[i], u=self.u[i],
-                     out=self.o_host[i])
+                     out=self.o_host[i], workspace=self.ws)
 
     def gemv_only(self, i):
-        self.lq.gemv(self.packed[i], self.s[i], self.u[i], out=self.o[i])
+        self.lq.gemv(self.packed[i], self.s[i], self.u[i], out=self.o[i], workspace=self.ws)
 
     @property
     def packed_bytes(self):

@@ -7,8 +7,9 @@ no fallback: if liblq.so is missing or cannot be loaded, import fails loudly.
     o = diag(s) . W_q . (blockdiag(M^T) . T^{-1} . a)
 
 Entry points (same names as include/lq.h, minus the `lq_` prefix):
-    lifted_dim, pack_signs, unpack_signs, lift_activations, gemv, gemm,
-    get_device_status
+    lifted_dim, pack_signs, unpack_signs, lift_activations,
+    lift_activations_kron, gemv_workspace_size, gemv, lift_gemv, gemm, encode,
+    get_device_status (lq_selftest_wait_timeout is reached through `lib`)
 """
 
 from __future__ import annotations
@@ -23,8 +24,8 @@ LQ_OK, LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_TIMEOUT = 0, 
 LQ_F32, LQ_BF16 = 0, 1
 
 SYMBOLS = ("lq_status_str", "lq_lifted_dim", "lq_pack_signs", "lq_unpack_signs", "lq_lift_activations",
-           "lq_lift_activations_kron", "lq_gemv", "lq_lift_gemv", "lq_gemm", "lq_encode",
-           "lq_selftest_wait_timeout", "lq_get_device_status")
+           "lq_lift_activations_kron", "lq_gemv_workspace_size", "lq_gemv", "lq_lift_gemv", "lq_gemm",
+           "lq_encode", "lq_selftest_wait_timeout", "lq_get_device_status")
 
 
 class LQError(RuntimeError):
@@ -50,10 +51,13 @@ def _load() -> ctypes.CDLL:
     lib.lq_lift_activations.argtypes = [p, i, i, i, p, i, p, i, i, p, i, i, p]
     lib.lq_lift_activations_kron.restype = i
     lib.lq_lift_activations_kron.argtypes = [p, i, i, i, p, p, i, p, i, p, p, i, i, p, i, i, p]
+    z = ctypes.c_size_t
+    lib.lq_gemv_workspace_size.restype = z
+    lib.lq_gemv_workspace_size.argtypes = [i, i, i]
     lib.lq_gemv.restype = i
-    lib.lq_gemv.argtypes = [p, p, i, i, p, i, p, p]
+    lib.lq_gemv.argtypes = [p, p, i, i, p, i, p, p, z, p]
     lib.lq_lift_gemv.restype = i
-    lib.lq_lift_gemv.argtypes = [p, i, i, i, p, i, p, i, i, p, p, i, i, p, p, p]
+    lib.lq_lift_gemv.argtypes = [p, i, i, i, p, i, p, i, i, p, p, i, i, p, p, p, z, p]
     lib.lq_gemm.restype = i
     lib.lq_encode.restype = i
     lib.lq_selftest_wait_timeout.restype = i
@@ -162,16 +166,45 @@ def lift_activations_kron(a, q1, q2, M, K, r1=None, r2=None, u_dtype="f32", out=
     return out
 
 
-def gemv(packed, s, u, out=None, stream=None):
-    """Decode: packed [out][K/32], s [out], u fp32 [batch][K] (batch <= 16) -> o fp32 [batch][out]."""
+def gemv_workspace_size(out_rows: int, K: int, batch: int) -> int:
+    """Bytes of device scratch lq_gemv / lq_lift_gemv need (0: shape not supported)."""
+    return int(lib.lq_gemv_workspace_size(out_rows, K, batch))
+
+
+def gemv_workspace(out_rows: int, K: int, batch: int, device=None):
+    """A device scratch tensor big enough for lq_gemv / lq_lift_gemv on this shape
+    (256-byte aligned: the caching allocator hands out 512-byte aligned blocks)."""
+    import torch
+    n = gemv_workspace_size(out_rows, K, batch)
+    if n == 0:
+        raise LQError(LQ_ERR_INVALID_ARG, "lq_gemv_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device if device is not None else "cuda")
+
+
+def _workspace(ws, out_rows, K, batch, device):
+    if ws is None:
+        ws = gemv_workspace(out_rows, K, batch, device)
+    _dev_tensor(ws, "workspace")
+    return ws
+
+
+def gemv(packed, s, u, out=None, workspace=None, stream=None):
+    """Decode: packed [out][K/32], s [out], u fp32 [batch][K] (batch <= 16) -> o fp32 [batch][out].
+
+    `workspace` (uint8 CUDA tensor of gemv_workspace_size bytes) is allocated
+    when not given; calls that share one must run on the same stream."""
     import torch
     _dev_tensor(packed, "packed")
+    _dev_tensor(s, "s")
     _dev_tensor(u, "u")
     rows = packed.shape[0]
     batch, K = u.shape
     if out is None:
         out = torch.empty((batch, rows), dtype=torch.float32, device=u.device)
-    _check(lib.lq_gemv(_ptr(packed), _ptr(s), rows, K, _ptr(u), batch, _ptr(out), _stream(stream)), "lq_gemv")
+    _dev_tensor(out, "out")
+    ws = _workspace(workspace, rows, K, batch, u.device)
+    _check(lib.lq_gemv(_ptr(packed), _ptr(s), rows, K, _ptr(u), batch, _ptr(out), _ptr(ws), ws.numel(),
+                       _stream(stream)), "lq_gemv")
     return out
 
 
@@ -181,7 +214,7 @@ def _dev_or_pinned(t, name):
     return t
 
 
-def lift_gemv(a, M, packed, s, K, tinv=None, u=None, out=None, stream=None):
+def lift_gemv(a, M, packed, s, K, tinv=None, u=None, out=None, workspace=None, stream=None):
     """Fused decode step: a [batch][in] (float32 or bfloat16) -> (u fp32 [batch][K], o fp32 [batch][out]).
 
     `a` and `out` may be pinned host tensors (zero-copy: the kernels read and
@@ -190,6 +223,7 @@ def lift_gemv(a, M, packed, s, K, tinv=None, u=None, out=None, stream=None):
     _dev_or_pinned(a, "a")
     _dev_tensor(M, "M")
     _dev_tensor(packed, "packed")
+    _dev_tensor(s, "s")
     batch, in_dim = a.shape
     d, D = M.shape
     rows = packed.shape[0]
@@ -203,8 +237,9 @@ def lift_gemv(a, M, packed, s, K, tinv=None, u=None, out=None, stream=None):
     tblk = 0 if tinv is None else int(tinv.shape[-1])
     if tinv is not None:
         _dev_tensor(tinv, "tinv")
+    ws = _workspace(workspace, rows, K, batch, M.device)
     _check(lib.lq_lift_gemv(_ptr(a), a_t, batch, in_dim, _ptr(tinv), tblk, _ptr(M), d, D, _ptr(packed), _ptr(s),
-                            rows, K, _ptr(u), _ptr(out), _stream(stream)), "lq_lift_gemv")
+                            rows, K, _ptr(u), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "lq_lift_gemv")
     return u, out
 
 
@@ -212,11 +247,13 @@ def gemm(packed, s, u, out=None, stream=None):
     """Prefill: packed [out][K/32], s [out], u bf16 [tokens][K] -> o fp32 [tokens][out]."""
     import torch
     _dev_tensor(packed, "packed")
+    _dev_tensor(s, "s")
     _dev_tensor(u, "u")
     rows = packed.shape[0]
     tokens, K = u.shape
     if out is None:
         out = torch.empty((tokens, rows), dtype=torch.float32, device=u.device)
+    _dev_tensor(out, "out")
     _check(lib.lq_gemm(_ptr(packed), _ptr(s), rows, K, _ptr(u), tokens, _ptr(out), _stream(stream)), "lq_gemm")
     return out
 

@@ -8,12 +8,32 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <initializer_list>
+
 #include "lq.h"
 #include "lq_internal.h"
 
 namespace {
 
 __device__ unsigned g_lq_status;
+__device__ unsigned g_lq_status_read;
+
+// Reads and clears the status word in one atomic step, so that a timeout a
+// kernel on another stream latches meanwhile is either returned or kept.
+__global__ void status_exchange_kernel() { g_lq_status_read = atomicExch(&g_lq_status, 0u); }
+
+// Makes `dev` current for its lifetime and restores the previous device.
+struct DeviceScope {
+    int prev = -1;
+    bool ok = false;
+    explicit DeviceScope(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) return;
+        ok = prev == dev || cudaSetDevice(dev) == cudaSuccess;
+    }
+    ~DeviceScope() {
+        if (ok && prev >= 0) cudaSetDevice(prev);
+    }
+};
 
 constexpr int kMaxDevices = 64;
 
@@ -41,6 +61,29 @@ bool device_addressable(const void* p) {
     }
     if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) return true;
     return at.type == cudaMemoryTypeHost && at.devicePointer == p;
+}
+
+// True if every non-null pointer is device-addressable (see above).
+bool all_addressable(std::initializer_list<const void*> ps) {
+    for (const void* p : ps)
+        if (p && !device_addressable(p)) return false;
+    return true;
+}
+
+// True if every non-null pointer is device or managed memory (host memory,
+// even page-locked, is refused: the kernels read these operands with TMA or
+// keep them in L2).
+bool all_device(std::initializer_list<const void*> ps) {
+    for (const void* p : ps) {
+        if (!p) continue;
+        cudaPointerAttributes at;
+        if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) return false;
+    }
+    return true;
 }
 
 // Device address of the status word on the current device (looked up once per device).
@@ -105,6 +148,7 @@ int lq_pack_signs(const int8_t* signs_pm1, int out, int K, uint32_t* packed, voi
     if (!signs_pm1 || !packed || !aligned16(signs_pm1) || !aligned16(packed)) return LQ_ERR_INVALID_ARG;
     if (out < 1 || K < 32 || K % 32 != 0) return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
+    if (!all_device({signs_pm1, packed})) return LQ_ERR_INVALID_ARG;
     return from_cuda(lq::launch_pack(signs_pm1, out, K, packed, static_cast<cudaStream_t>(stream)));
 }
 
@@ -112,6 +156,7 @@ int lq_unpack_signs(const uint32_t* packed, int out, int K, int8_t* signs_pm1, v
     if (!signs_pm1 || !packed || !aligned16(signs_pm1) || !aligned16(packed)) return LQ_ERR_INVALID_ARG;
     if (out < 1 || K < 32 || K % 32 != 0) return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
+    if (!all_device({packed, signs_pm1})) return LQ_ERR_INVALID_ARG;
     return from_cuda(lq::launch_unpack(packed, out, K, signs_pm1, static_cast<cudaStream_t>(stream)));
 }
 
@@ -125,6 +170,10 @@ int lq_lift_activations(const void* a, int a_dtype, int batch, int in, const flo
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
     if (tinv && (tblk < 1 || tblk > 256 || in % tblk != 0)) return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
+    const int sm = is_sm100();
+    if (sm < 0) return LQ_ERR_CUDA;
+    if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    if (!all_device({a, tinv, M, u})) return LQ_ERR_INVALID_ARG;
     int err = LQ_OK;
     unsigned* status = status_word(&err);
     if (!status) return err;
@@ -150,6 +199,7 @@ int lq_lift_activations_kron(const void* a, int a_dtype, int batch, int in, cons
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    if (!all_device({a, r1, q1, q2, r2, M, u})) return LQ_ERR_INVALID_ARG;
     return from_cuda(lq::launch_lift_kron(a, a_dtype == LQ_BF16, batch, in, r1, q1, n1, q2, n2, r2, M, d, D, u,
                                           u_dtype == LQ_BF16, K, static_cast<cudaStream_t>(stream)));
 }
@@ -165,6 +215,7 @@ int lq_encode(const float* w, int rows, int in, const float* M, int d, int D, ui
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    if (!all_device({w, M, packed, err})) return LQ_ERR_INVALID_ARG;
     return from_cuda(lq::launch_encode(w, rows, in, M, d, D, packed, K, err, static_cast<cudaStream_t>(stream)));
 }
 
@@ -180,44 +231,57 @@ int lq_selftest_wait_timeout(unsigned limit_us, void* stream) {
     return from_cuda(lq::launch_selftest_wait_timeout(limit_us, status, static_cast<cudaStream_t>(stream)));
 }
 
+size_t lq_gemv_workspace_size(int out, int K, int batch) {
+    if (out < 1 || K < 32 || K % 32 != 0 || batch < 1 || batch > 16) return 0;
+    return lq::gemv_workspace_size(out, K, batch);
+}
+
 int lq_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u, int batch, float* o,
-            void* stream) {
-    if (!packed || !s || !u || !o) return LQ_ERR_INVALID_ARG;
+            void* workspace, size_t workspace_bytes, void* stream) {
+    if (!packed || !s || !u || !o || !workspace) return LQ_ERR_INVALID_ARG;
     if (!aligned16(packed) || !aligned16(s) || !aligned16(u) || !aligned16(o)) return LQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LQ_ERR_INVALID_ARG;
     if (out < 1 || K < 32 || K % 32 != 0 || batch < 1 || batch > 16) return LQ_ERR_INVALID_ARG;
-    if (!lq::gemv_supported(out, K, batch)) return LQ_ERR_INVALID_ARG;
+    const size_t need = lq::gemv_workspace_size(out, K, batch);
+    if (need == 0 || workspace_bytes < need) return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    if (!all_device({packed, s, u, o, workspace})) return LQ_ERR_INVALID_ARG;
     int err = LQ_OK;
     unsigned* status = status_word(&err);
     if (!status) return err;
-    return from_cuda(lq::launch_gemv(packed, s, out, K, u, batch, o, status, static_cast<cudaStream_t>(stream)));
+    return from_cuda(lq::launch_gemv(packed, s, out, K, u, batch, o, workspace, status,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 int lq_lift_gemv(const void* a, int a_dtype, int batch, int in, const float* tinv, int tblk, const float* M, int d,
-                 int D, const uint32_t* packed, const float* s, int out, int K, float* u, float* o, void* stream) {
-    if (!a || !M || !u || !packed || !s || !o) return LQ_ERR_INVALID_ARG;
+                 int D, const uint32_t* packed, const float* s, int out, int K, float* u, float* o,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+    if (!a || !M || !u || !packed || !s || !o || !workspace) return LQ_ERR_INVALID_ARG;
     if (!aligned16(a) || !aligned16(M) || !aligned16(u) || !aligned16(packed) || !aligned16(s) || !aligned16(o))
         return LQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LQ_ERR_INVALID_ARG;
     if (tinv && !aligned16(tinv)) return LQ_ERR_INVALID_ARG;
     if (a_dtype != LQ_F32 && a_dtype != LQ_BF16) return LQ_ERR_INVALID_ARG;
     if (batch < 1 || batch > 16 || in < 1 || d < 1 || d > 64 || D < 1 || D > 256 || d * D > 4096)
         return LQ_ERR_INVALID_ARG;
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
     if (tinv && (tblk < 1 || tblk > 256 || in % tblk != 0)) return LQ_ERR_INVALID_ARG;
-    if (out < 1 || !lq::gemv_supported(out, K, batch)) return LQ_ERR_INVALID_ARG;
+    if (out < 1) return LQ_ERR_INVALID_ARG;
+    const size_t need = lq::gemv_workspace_size(out, K, batch);
+    if (need == 0 || workspace_bytes < need) return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
-    if (!device_addressable(a) || !device_addressable(o)) return LQ_ERR_INVALID_ARG;
+    if (!all_addressable({a, o}) || !all_device({tinv, M, packed, s, u, workspace})) return LQ_ERR_INVALID_ARG;
     int err = LQ_OK;
     unsigned* status = status_word(&err);
     if (!status) return err;
     return from_cuda(lq::launch_lift_gemv(a, a_dtype == LQ_BF16, batch, in, tinv, tblk, M, d, D, packed, s, out, K, u,
-                                          o, status, static_cast<cudaStream_t>(stream)));
+                                          o, workspace, status, static_cast<cudaStream_t>(stream)));
 }
 
 int lq_gemm(const uint32_t* packed, const float* s, int out, int K, const uint16_t* u_bf16, int tokens, float* o,
@@ -229,6 +293,7 @@ int lq_gemm(const uint32_t* packed, const float* s, int out, int K, const uint16
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    if (!all_device({packed, s, u_bf16, o})) return LQ_ERR_INVALID_ARG;
     int err = LQ_OK;
     unsigned* status = status_word(&err);
     if (!status) return err;
@@ -237,13 +302,18 @@ int lq_gemm(const uint32_t* packed, const float* s, int out, int K, const uint16
 
 int lq_get_device_status(void* stream) {
     if (fault_is("timeout")) return LQ_ERR_TIMEOUT;
-    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return LQ_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int dev = 0;
+    if (cudaStreamGetDevice(st, &dev) != cudaSuccess) return LQ_ERR_CUDA;
+    DeviceScope scope(dev);  // the status word of the stream's device
+    if (!scope.ok) return LQ_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return LQ_ERR_CUDA;
+    status_exchange_kernel<<<1, 1, 0, st>>>();
+    if (cudaGetLastError() != cudaSuccess) return LQ_ERR_CUDA;
     unsigned v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_lq_status, sizeof(v)) != cudaSuccess) return LQ_ERR_CUDA;
-    if (v) {
-        const unsigned zero = 0;
-        if (cudaMemcpyToSymbol(g_lq_status, &zero, sizeof(zero)) != cudaSuccess) return LQ_ERR_CUDA;
-    }
+    if (cudaMemcpyFromSymbolAsync(&v, g_lq_status_read, sizeof(v), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return LQ_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return LQ_ERR_CUDA;
     return (v & LQ_DEV_TIMEOUT) ? LQ_ERR_TIMEOUT : LQ_OK;
 }
 

@@ -45,19 +45,35 @@ cudaError_t launch_encode(const float* w, int rows, int in, const float* M, int 
 // Self-test of the bounded waits: one wait that nothing completes, limit_us long.
 cudaError_t launch_selftest_wait_timeout(unsigned limit_us, unsigned* status, cudaStream_t st);
 
-// Decode GEMV (integer tensor cores; u quantized per CTA). `status` is the
-// device status word that bounded waits report to.
-// Whether the GEMV's launch plan fits in shared memory for this shape (each CTA
-// keeps 64-bit partial sums for its rows, so very large `out` does not fit).
-bool gemv_supported(int out, int K, int batch);
+// Decode GEMV (lq_decode.h): the quantizer writes u's digit planes into the
+// caller's workspace, then the mma.sync kernel (batch 1..2, or when the
+// tcgen05 plan does not fit) or the tcgen05 kernel (batch >= 3) contracts.
+// `status` is the device status word that bounded waits report to.
+// gemv_workspace_size is 0 when no launch plan fits the shape (each mma.sync
+// CTA keeps 64-bit partial sums for its rows, so a very large `out` does not fit).
+size_t gemv_workspace_size(int out, int K, int batch);
 cudaError_t launch_gemv(const uint32_t* packed, const float* s, int out, int K, const float* u,
-                        int batch, float* o, unsigned* status, cudaStream_t st);
+                        int batch, float* o, void* ws, unsigned* status, cudaStream_t st);
 
-// Decode step: the lift into u, then the GEMV (a programmatic dependent of the
-// lift, so its prologue overlaps the lift where both fit on an SM).
+// Decode step: the lift into u, the quantizer, then the contraction, each a
+// programmatic dependent of the one before.
 cudaError_t launch_lift_gemv(const void* a, bool a_bf16, int batch, int in, const float* tinv, int tblk,
                              const float* M, int d, int D, const uint32_t* packed, const float* s, int out, int K,
-                             float* u, float* o, unsigned* status, cudaStream_t st);
+                             float* u, float* o, void* ws, unsigned* status, cudaStream_t st);
+
+struct DecodePlan;
+// The quantizers (lq_quant.cu): 32-bit fixed point for the mma.sync kernel
+// (it also clears `nzero` words at `zero`), block-scaled e2m1 digits for the
+// tcgen05 kernel (it also clears the kernel's group counters).
+cudaError_t launch_quant(const float* u, const DecodePlan& p, void* ws, unsigned* zero, int nzero, cudaStream_t st);
+cudaError_t launch_quant_mx(const float* u, const DecodePlan& p, void* ws, cudaStream_t st);
+// The tcgen05 contraction (lq_gemv_tc.cu): plan_tc fills the tc_* fields and
+// returns whether the shape takes that kernel; tc_slot_bytes is the size of its
+// partial-sum slots in the workspace.
+bool plan_tc(DecodePlan& p);
+size_t tc_slot_bytes(const DecodePlan& p);
+cudaError_t launch_gemv_tc(const uint32_t* packed, const float* s, const DecodePlan& p, float* o, uint8_t* ws,
+                           unsigned* status, cudaStream_t st);
 
 // Prefill GEMM on tcgen05. `status` is the device status word.
 cudaError_t launch_gemm(const uint32_t* packed, const float* s, int out, int K,

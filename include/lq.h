@@ -13,7 +13,9 @@
  * Conventions shared by every call
  *  - All tensor pointers are caller-owned DEVICE memory (lq_lift_gemv's `a`
  *    and `o` may also be mapped page-locked host memory), 16-byte aligned,
- *    densely packed row-major. The library frees nothing and keeps no pointer.
+ *    densely packed row-major; the compute calls check this with
+ *    cudaPointerGetAttributes and refuse host memory with LQ_ERR_INVALID_ARG.
+ *    The library frees nothing and keeps no pointer.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
  *    stream-ordered and asynchronous: they return after enqueueing work.
  *  - Argument checks are synchronous and happen before any launch; a call
@@ -33,6 +35,7 @@
 #ifndef LQ_H
 #define LQ_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -112,8 +115,11 @@ LQ_API int lq_encode(const float* w, int rows, int in, const float* M, int d, in
  * into three bf16 parts (24 significant bits, fp32 accumulation): the same
  * accuracy class as the fp32 kernels. Bounded waits inside that kernel report
  * LQ_ERR_TIMEOUT through lq_get_device_status. The decode kernel is launched as
- * a programmatic dependent of the preceding kernel on the stream and waits for
- * it before reading a. */
+ * a programmatic dependent of the preceding kernel on the stream: it may read
+ * tinv and M before that kernel completes (so that this overlaps it), and waits
+ * for it before reading a. Do not let the preceding kernel write tinv or M.
+ * Every pointer must be device memory. Requires an sm_100 device (else
+ * LQ_ERR_UNSUPPORTED). */
 LQ_API int lq_lift_activations(const void* a, int a_dtype, int batch, int in,
                         const float* tinv, int tblk,
                         const float* M, int d, int D,
@@ -144,43 +150,58 @@ LQ_API int lq_lift_activations_kron(const void* a, int a_dtype, int batch, int i
                                     const float* r2, const float* M, int d, int D,
                                     void* u, int u_dtype, int K, void* stream);
 
+/* Workspace bytes lq_gemv and lq_lift_gemv need for (out, K, batch); 0 if the
+ * arguments are invalid or no launch plan fits the shape. Host only; the size
+ * depends on the device's SM count only through the plan, so query it on the
+ * device that will run the call. */
+LQ_API size_t lq_gemv_workspace_size(int out, int K, int batch);
+
 /* Decode 1-bit GEMV, batch 1..16 (the +-1 by float matmul of "Key designs" 4):
  *   o[c][r] = s[r] * sum_k sigma[r][k] * u[c][k],  sigma = +1 if bit set else -1
  *   packed : uint32 [out][K/32]; s : fp32 [out]; u : fp32 [batch][K]
  *   o      : fp32 [batch][out] (written)
  *   out >= 1, K >= 32, K % 32 == 0, 1 <= batch <= 16
- * u is converted per K-part and column to 24-bit fixed point (error <= 2^-22 of
- * the part's largest |u|); the sign contraction itself is exact integer
- * arithmetic, so the result is within ~1e-6 relative (Frobenius) of the exact
- * value. Deterministic. Needs no scratch memory. Each CTA keeps 64-bit partial
- * sums for its rows in shared memory, which bounds `out` (about 3.1 million rows
- * for K in the tens of thousands on a 148-SM B200); larger shapes return
- * LQ_ERR_INVALID_ARG. Requires an sm_100 device (else LQ_ERR_UNSUPPORTED). */
+ *   workspace : caller-owned device scratch of at least
+ *               lq_gemv_workspace_size(out, K, batch) bytes, 256-byte aligned;
+ *               its contents need no initialization and are overwritten.
+ * Arithmetic: each column of u is converted once per call to 32-bit fixed
+ * point with one power-of-two scale (an element's error is at most 2^-31 of the
+ * column's largest |u|), and the sign contraction is exact integer arithmetic,
+ * so the result is within ~1e-7 relative (Frobenius) of the exact value, and
+ * exactly equal to it when u holds small integers. Non-finite activations
+ * propagate as in an exact IEEE sum: a column holding a NaN gives NaN; a column
+ * holding +-Inf gives, per row, +-Inf or NaN by the signs of its Inf terms.
+ * Deterministic. Batches of three or more read every weight once (tcgen05);
+ * one or two columns run on mma.sync. Calls that share a workspace must be
+ * ordered (the same stream): overlapping calls race on it. Every pointer must
+ * be device memory. The call's first kernel waits for the preceding kernel on
+ * the stream before it reads anything. Requires an sm_100 device (else
+ * LQ_ERR_UNSUPPORTED). */
 LQ_API int lq_gemv(const uint32_t* packed, const float* s, int out, int K,
-            const float* u, int batch, float* o, void* stream);
+            const float* u, int batch, float* o, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Decode step in one call: lq_lift_activations followed by lq_gemv (the small
  * matmul T* a, then the 1-bit x float matmul and diag(s) -- "Key designs" 4),
  * with the arguments of both calls:
  *   a, a_dtype, batch, in, tinv, tblk, M, d, D, K : as lq_lift_activations
- *   packed, s, out                               : as lq_gemv
+ *   packed, s, out, workspace, workspace_bytes     : as lq_gemv
  *   u : fp32 [batch][K] (written: the lifted activations)
  *   o : fp32 [batch][out] (written); 1 <= batch <= 16
- * Results are exactly those of the two calls; the GEMV is launched as a
- * programmatic dependent of the lift, so its setup and first weight requests
- * overlap the lift.
+ * Results are exactly those of the two calls; the kernels are chained as
+ * programmatic dependents, so each one's setup overlaps the one before.
  * Zero-copy decode: `a` and `o` (only these two) may instead be page-locked
  * host memory that the device addresses at the same pointer (with unified
  * addressing, any cudaHostAlloc / cudaMallocHost buffer). The lift then loads
  * the activations, and the GEMV stores the outputs, across the host link
  * itself, so a step from host buffers needs no separate copies; the results
- * are identical. The call checks both pointers with cudaPointerGetAttributes
- * and returns LQ_ERR_INVALID_ARG for pageable or unmapped host memory. The
- * host must not touch `a` or `o` until the stream has passed the call.
- * Requires an sm_100 device (else LQ_ERR_UNSUPPORTED). */
+ * are identical. The call checks every pointer with cudaPointerGetAttributes
+ * and returns LQ_ERR_INVALID_ARG for pageable or unmapped host memory (and for
+ * host memory anywhere but `a` and `o`). The host must not touch `a` or `o`
+ * until the stream has passed the call. Requires an sm_100 device (else
+ * LQ_ERR_UNSUPPORTED). */
 LQ_API int lq_lift_gemv(const void* a, int a_dtype, int batch, int in, const float* tinv, int tblk,
                         const float* M, int d, int D, const uint32_t* packed, const float* s, int out, int K,
-                        float* u, float* o, void* stream);
+                        float* u, float* o, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Prefill 1-bit GEMM on the tensor cores (tcgen05, bf16 operands, fp32 accumulate):
  *   o[t][r] = s[r] * sum_k sigma[r][k] * u[t][k]
@@ -200,9 +221,11 @@ LQ_API int lq_gemm(const uint32_t* packed, const float* s, int out, int K,
  * sm_100 device (else LQ_ERR_UNSUPPORTED). */
 LQ_API int lq_selftest_wait_timeout(unsigned limit_us, void* stream);
 
-/* Synchronizes `stream`, then returns and clears the device status word of the
- * current device: LQ_OK, or LQ_ERR_TIMEOUT if a kernel gave up a bounded wait
- * since the last call. Returns LQ_ERR_CUDA if the synchronize fails. */
+/* Synchronizes `stream`, then reads and clears, in one atomic exchange on the
+ * device, the status word of the stream's device: LQ_OK, or LQ_ERR_TIMEOUT if a
+ * kernel there gave up a bounded wait since the last call. A timeout latched
+ * meanwhile by a kernel on another stream is either returned or kept for the
+ * next call. Returns LQ_ERR_CUDA if a CUDA call fails. */
 LQ_API int lq_get_device_status(void* stream);
 
 #ifdef __cplusplus

@@ -49,6 +49,8 @@ def test_lifted_dim_matches_oracle_closed_form():
 
 P = 0x100000  # a 16-byte-aligned fake address; never dereferenced (validation fails first)
 MIS = P + 4   # misaligned
+W = 0x200000  # a 256-byte-aligned fake workspace address
+BIG = 1 << 40  # workspace bytes: more than any shape needs
 
 
 def _c(v):
@@ -61,21 +63,24 @@ def _c(v):
     ("pack out<1", "lq_pack_signs", [_c(P), 0, 32, _c(P), None]),
     ("pack misaligned", "lq_pack_signs", [_c(MIS), 4, 32, _c(P), None]),
     ("unpack null", "lq_unpack_signs", [_c(P), 4, 32, None, None]),
-    ("gemv batch 0", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 0, _c(P), None]),
-    ("gemv batch 17", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 17, _c(P), None]),
-    ("gemv K%32", "lq_gemv", [_c(P), _c(P), 8, 40, _c(P), 1, _c(P), None]),
-    ("gemv misaligned u", "lq_gemv", [_c(P), _c(P), 8, 64, _c(MIS), 1, _c(P), None]),
-    ("gemv null s", "lq_gemv", [_c(P), None, 8, 64, _c(P), 1, _c(P), None]),
+    ("gemv batch 0", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 0, _c(P), _c(W), BIG, None]),
+    ("gemv batch 17", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 17, _c(P), _c(W), BIG, None]),
+    ("gemv K%32", "lq_gemv", [_c(P), _c(P), 8, 40, _c(P), 1, _c(P), _c(W), BIG, None]),
+    ("gemv misaligned u", "lq_gemv", [_c(P), _c(P), 8, 64, _c(MIS), 1, _c(P), _c(W), BIG, None]),
+    ("gemv null workspace", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 1, _c(P), None, BIG, None]),
+    ("gemv workspace misaligned", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 1, _c(P), _c(W + 16), BIG, None]),
+    ("gemv workspace too small", "lq_gemv", [_c(P), _c(P), 8, 64, _c(P), 1, _c(P), _c(W), 16, None]),
+    ("gemv null s", "lq_gemv", [_c(P), None, 8, 64, _c(P), 1, _c(P), _c(W), BIG, None]),
     ("lift_gemv batch 17", "lq_lift_gemv", [_c(P), 0, 17, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 8, 1536,
-                                            _c(P), _c(P), None]),
+                                            _c(P), _c(P), _c(W), BIG, None]),
     ("lift_gemv K mismatch", "lq_lift_gemv", [_c(P), 0, 1, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 8, 1504,
-                                              _c(P), _c(P), None]),
+                                              _c(P), _c(P), _c(W), BIG, None]),
     ("lift_gemv null o", "lq_lift_gemv", [_c(P), 0, 1, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 8, 1536,
-                                          _c(P), None, None]),
+                                          _c(P), None, _c(W), BIG, None]),
     ("lift_gemv misaligned u", "lq_lift_gemv", [_c(P), 0, 1, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 8, 1536,
-                                                _c(MIS), _c(P), None]),
+                                                _c(MIS), _c(P), _c(W), BIG, None]),
     ("lift_gemv out 0", "lq_lift_gemv", [_c(P), 0, 1, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 0, 1536,
-                                         _c(P), _c(P), None]),
+                                         _c(P), _c(P), _c(W), BIG, None]),
     ("gemm tokens 0", "lq_gemm", [_c(P), _c(P), 8, 64, _c(P), 0, _c(P), None]),
     ("gemm K<32", "lq_gemm", [_c(P), _c(P), 8, 0, _c(P), 4, _c(P), None]),
     ("gemm null o", "lq_gemm", [_c(P), _c(P), 8, 64, _c(P), 4, None, None]),
@@ -142,19 +147,24 @@ def test_fault_injection_launch(monkeypatch):
     import bit_lifted_gemm_b200 as lq
     monkeypatch.setenv("LQ_FAULT", "launch")
     assert lq.lib.lq_pack_signs(_c(P), 4, 32, _c(P), None) == lq.LQ_ERR_CUDA
-    assert lq.lib.lq_gemv(_c(P), _c(P), 8, 64, _c(P), 1, _c(P), None) == lq.LQ_ERR_CUDA
+    assert lq.lib.lq_gemv(_c(P), _c(P), 8, 64, _c(P), 1, _c(P), _c(W), BIG, None) == lq.LQ_ERR_CUDA
     assert lq.lib.lq_gemm(_c(P), _c(P), 8, 64, _c(P), 4, _c(P), None) == lq.LQ_ERR_CUDA
     assert lq.lib.lq_encode(_c(P), 4, 40, _c(P), 4, 12, _c(P), 128, None, None) == lq.LQ_ERR_CUDA
-    assert lq.lib.lq_gemv(_c(P), _c(P), 8, 64, _c(P), 0, _c(P), None) == lq.LQ_ERR_INVALID_ARG
+    assert lq.lib.lq_gemv(_c(P), _c(P), 8, 64, _c(P), 0, _c(P), _c(W), BIG, None) == lq.LQ_ERR_INVALID_ARG
 
 
 def test_gemv_rejects_rows_beyond_the_plan():
-    """Row counts whose per-CTA partial sums cannot fit in shared memory are
-    refused before any launch (a 2^24-row exhaustive codebook, for instance)."""
+    """Row lengths that are not a multiple of four words run on the mma.sync
+    kernel, whose CTAs keep 64-bit partial sums for their rows in shared memory;
+    row counts beyond that plan are refused before any launch (a 2^24-row
+    exhaustive codebook, for instance). The tensor-core plan for K % 128 == 0
+    has no such bound."""
     import bit_lifted_gemm_b200 as lq
-    assert lq.lib.lq_gemv(_c(P), _c(P), 1 << 24, 32, _c(P), 1, _c(P), None) == lq.LQ_ERR_INVALID_ARG
-    assert lq.lib.lq_lift_gemv(_c(P), 0, 1, 640, None, 0, _c(P), 10, 24, _c(P), _c(P), 1 << 24, 1536,
-                               _c(P), _c(P), None) == lq.LQ_ERR_INVALID_ARG
+    assert lq.gemv_workspace_size(1 << 24, 32, 1) == 0
+    assert lq.lib.lq_gemv(_c(P), _c(P), 1 << 24, 32, _c(P), 1, _c(P), _c(W), BIG, None) == lq.LQ_ERR_INVALID_ARG
+    assert lq.lib.lq_lift_gemv(_c(P), 0, 1, 650, None, 0, _c(P), 10, 24, _c(P), _c(P), 1 << 24, 1568,
+                               _c(P), _c(P), _c(W), BIG, None) == lq.LQ_ERR_INVALID_ARG
+    assert lq.gemv_workspace_size(1 << 24, 1536, 1) > 0
 
 
 def test_gemv_plan_fits_every_configured_layer(monkeypatch):
@@ -168,5 +178,10 @@ def test_gemv_plan_fits_every_configured_layer(monkeypatch):
         if cfg.kind == "prefill":
             continue
         for batch in (1, 2, 4, 8, 16):
-            rc = lq.lib.lq_gemv(_c(P), _c(P), cfg.out, cfg.K, _c(P), batch, _c(P), None)
+            ws = lq.gemv_workspace_size(cfg.out, cfg.K, batch)
+            assert ws > 0, (cfg.name, batch)
+            rc = lq.lib.lq_gemv(_c(P), _c(P), cfg.out, cfg.K, _c(P), batch, _c(P), _c(W), ws, None)
             assert rc == lq.LQ_ERR_CUDA, (cfg.name, batch)
+            # one byte short of the workspace the plan needs is refused
+            rc = lq.lib.lq_gemv(_c(P), _c(P), cfg.out, cfg.K, _c(P), batch, _c(P), _c(W), ws - 1, None)
+            assert rc == lq.LQ_ERR_INVALID_ARG, (cfg.name, batch)

@@ -402,10 +402,11 @@ def test_fused_step_rejects_pageable_host(lq):
     o = torch.empty((1, L.cfg.out), dtype=torch.float32, device="cuda")
     M, pk, s = dev(L.M), dev(L.packed), dev(L.s)
     d, D = L.M.shape
+    ws = lq.gemv_workspace(L.cfg.out, L.cfg.K, 1)
     rc = lq.lib.lq_lift_gemv(ctypes.c_void_p(a_p.data_ptr()), lq.LQ_F32, 1, L.cfg.in_dim, None, 0,
                              ctypes.c_void_p(M.data_ptr()), d, D, ctypes.c_void_p(pk.data_ptr()),
                              ctypes.c_void_p(s.data_ptr()), L.cfg.out, L.cfg.K, ctypes.c_void_p(u.data_ptr()),
-                             ctypes.c_void_p(o.data_ptr()), None)
+                             ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(ws.data_ptr()), ws.numel(), None)
     assert rc == lq.LQ_ERR_INVALID_ARG
 
 
@@ -472,8 +473,9 @@ def test_prefill_lq24_10_full_size_sampled(lq):
     assert rel_err(o[np.ix_(toks, rows)], want) <= 5e-3
 
 
-@pytest.mark.parametrize("D", [16, 24])
+@pytest.mark.parametrize("D", [16, 19, 20, 22, 24])
 def test_sweep_prefill_b64(lq, D):
+    """Every configured bit-width at 64 tokens (the shapes the benchmark times)."""
     L = make_layer(CONFIGS[f"sweep_lq{D}_8"], 64)
     u = _gpu_u(lq, L, "bf16")
     o = host(lq.gemm(dev(L.packed), dev(L.s), u))
