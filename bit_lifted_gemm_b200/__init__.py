@@ -20,12 +20,13 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblq.so")
 
-LQ_OK, LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_TIMEOUT = 0, 1, 2, 3, 4
+LQ_OK, LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_TIMEOUT, LQ_ERR_TOO_LARGE = 0, 1, 2, 3, 4, 5
 LQ_F32, LQ_BF16 = 0, 1
+GEMV_NOALLOC_SCRATCH_BYTES = 4 << 20  # LQ_GEMV_NOALLOC_SCRATCH_BYTES of include/lq.h
 
 SYMBOLS = ("lq_status_str", "lq_lifted_dim", "lq_pack_signs", "lq_unpack_signs", "lq_lift_activations",
-           "lq_lift_activations_kron", "lq_gemv_workspace_size", "lq_gemv", "lq_lift_gemv", "lq_gemm",
-           "lq_encode", "lq_selftest_wait_timeout", "lq_get_device_status")
+           "lq_lift_activations_kron", "lq_gemv_workspace_size", "lq_gemv", "lq_gemv_noalloc", "lq_lift_gemv",
+           "lq_gemm", "lq_encode", "lq_selftest_wait_timeout", "lq_get_device_status")
 
 
 class LQError(RuntimeError):
@@ -56,6 +57,8 @@ def _load() -> ctypes.CDLL:
     lib.lq_gemv_workspace_size.argtypes = [i, i, i]
     lib.lq_gemv.restype = i
     lib.lq_gemv.argtypes = [p, p, i, i, p, i, p, p, z, p]
+    lib.lq_gemv_noalloc.restype = i
+    lib.lq_gemv_noalloc.argtypes = [p, p, i, i, p, i, p, p]
     lib.lq_lift_gemv.restype = i
     lib.lq_lift_gemv.argtypes = [p, i, i, i, p, i, p, i, i, p, p, i, i, p, p, p, z, p]
     lib.lq_gemm.restype = i

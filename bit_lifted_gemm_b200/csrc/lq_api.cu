@@ -133,6 +133,7 @@ const char* lq_status_str(int status) {
         case LQ_ERR_UNSUPPORTED: return "LQ_ERR_UNSUPPORTED";
         case LQ_ERR_CUDA: return "LQ_ERR_CUDA";
         case LQ_ERR_TIMEOUT: return "LQ_ERR_TIMEOUT";
+        case LQ_ERR_TOO_LARGE: return "LQ_ERR_TOO_LARGE";
         default: return "LQ_ERR_UNKNOWN";
     }
 }
@@ -315,6 +316,62 @@ int lq_get_device_status(void* stream) {
         return LQ_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return LQ_ERR_CUDA;
     return (v & LQ_DEV_TIMEOUT) ? LQ_ERR_TIMEOUT : LQ_OK;
+}
+
+// ---------------------------------------------------------------- decode GEMV without allocation
+//
+// For callers that cannot allocate device memory (see lq.h): the scratch that
+// lq_gemv takes as a workspace lives in this fixed device array instead. Every
+// device that loads the library holds it until the process exits. Its address is
+// looked up once per device, with that device current; host code must never hand
+// the array's name itself to a kernel (on the host it is only a stand-in).
+
+}  // extern "C"
+
+static __device__ __align__(256) uint8_t g_lq_static_scratch[LQ_GEMV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of the static scratch on the current device, or null on error.
+void* static_scratch() {
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return nullptr;
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_lq_static_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int lq_gemv_noalloc(const uint32_t* packed, const float* s, int out, int K, const float* u, int batch, float* o,
+                    void* stream) {
+    if (!packed || !s || !u || !o) return LQ_ERR_INVALID_ARG;
+    if (!aligned16(packed) || !aligned16(s) || !aligned16(u) || !aligned16(o)) return LQ_ERR_INVALID_ARG;
+    if (out < 1 || K < 32 || K % 32 != 0 || batch < 1 || batch > 16) return LQ_ERR_INVALID_ARG;
+    const size_t need = lq::gemv_workspace_size(out, K, batch);
+    if (need == 0) return LQ_ERR_INVALID_ARG;
+    if (need > LQ_GEMV_NOALLOC_SCRATCH_BYTES) return LQ_ERR_TOO_LARGE;
+    if (fault_is("launch")) return LQ_ERR_CUDA;
+    const int sm = is_sm100();
+    if (sm < 0) return LQ_ERR_CUDA;
+    if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    if (!all_device({packed, s, u, o})) return LQ_ERR_INVALID_ARG;
+    void* scratch = static_scratch();
+    if (!scratch) return LQ_ERR_CUDA;
+    int err = LQ_OK;
+    unsigned* status = status_word(&err);
+    if (!status) return err;
+    return from_cuda(lq::launch_gemv(packed, s, out, K, u, batch, o, scratch, status,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -53,7 +53,8 @@ typedef enum {
     LQ_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or dtype; nothing launched */
     LQ_ERR_UNSUPPORTED = 2,  /* valid but not supported on this device (needs sm_100) */
     LQ_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
-    LQ_ERR_TIMEOUT = 4       /* a device-side bounded wait expired (from lq_get_device_status) */
+    LQ_ERR_TIMEOUT = 4,      /* a device-side bounded wait expired (from lq_get_device_status) */
+    LQ_ERR_TOO_LARGE = 5     /* the shape needs more scratch than lq_gemv_noalloc's fixed array holds */
 } lq_status;
 
 typedef enum { LQ_F32 = 0, LQ_BF16 = 1 } lq_dtype;
@@ -202,6 +203,34 @@ LQ_API int lq_gemv(const uint32_t* packed, const float* s, int out, int K,
 LQ_API int lq_lift_gemv(const void* a, int a_dtype, int batch, int in, const float* tinv, int tblk,
                         const float* M, int d, int D, const uint32_t* packed, const float* s, int out, int K,
                         float* u, float* o, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Decode GEMV that allocates nothing: lq_gemv with the same arguments and the
+ * same results, minus the workspace. (The paper has no counterpart; this is a
+ * service of the library.) Some callers cannot call cudaMalloc or own scratch
+ * buffers: code that runs while a stream is being captured into a CUDA graph
+ * (allocation there is not allowed or would be baked into the graph), serving
+ * loops whose memory pool is fixed up front and may not grow (cudaMalloc can
+ * also synchronize the device, stalling every stream), and plug-ins or hooks
+ * that only receive tensors from their host framework. For them the scratch
+ * lives in a fixed device array of LQ_GEMV_NOALLOC_SCRATCH_BYTES inside the
+ * library, which every GPU that loads the library keeps until the process
+ * exits.
+ *   Sizes: shapes whose lq_gemv_workspace_size exceeds that array return
+ *   LQ_ERR_TOO_LARGE before any launch (every configured decode layer fits at
+ *   batches up to eight; the widest batches of large layers need lq_gemv).
+ *   Sharing: every call on a device uses the same array, and the array keeps
+ *   the previous call's contents (each call rewrites all it reads, so nothing
+ *   needs clearing). Calls that can overlap on the GPU -- on different streams
+ *   without ordering, or from several host threads -- race on it: issue them in
+ *   one stream order.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before capturing any stream.
+ *   Allocation: none (no cudaMalloc, cudaFree or allocating library routine).
+ * Requires an sm_100 device (else LQ_ERR_UNSUPPORTED). */
+#define LQ_GEMV_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+LQ_API int lq_gemv_noalloc(const uint32_t* packed, const float* s, int out, int K,
+                           const float* u, int batch, float* o, void* stream);
 
 /* Prefill 1-bit GEMM on the tensor cores (tcgen05, bf16 operands, fp32 accumulate):
  *   o[t][r] = s[r] * sum_k sigma[r][k] * u[t][k]
