@@ -72,11 +72,15 @@ __host__ __device__ inline int plane_pitch(int words) {
 constexpr int kMxPlanes = 7;
 constexpr int kMxQWords = 8;  // words of one column per quantizer CTA (one per warp)
 
-// Per-word info word (binfo): bits 0..8 the biased exponent E + kMxBias (0: the
-// word is all zero; E runs from -148 for the smallest subnormal to 128), bit 9
-// a NaN in the word, bit 10 an Inf, bits 16..21 the number of +-Inf elements.
-// Per-CTA column summary: bits 0..8 the largest biased exponent of its finite
-// words, bit 9 any NaN, bit 10 any Inf, bits 16..31 the number of +-Inf elements.
+// A word's info (inside the quantizer): bits 0..8 the biased exponent E + kMxBias
+// (0: the word is all zero; E runs from -148 for the smallest subnormal to 128),
+// bit 9 a NaN in the word, bit 10 an Inf, bits 16..21 the number of +-Inf
+// elements. Per quantizer CTA (kMxQWords words of one column) the workspace keeps
+// a summary: bits 0..8 the largest biased exponent E_loc of its finite words,
+// bit 9 any NaN, bit 10 any Inf, bits 16..31 the number of +-Inf elements; and
+// per word one delta byte: min(127, E_loc - E) (127 for all-zero and NaN
+// words), bit 7 set for a word holding +-Inf. The contraction rebuilds each
+// scale exponent from them with byte-wise saturating arithmetic.
 constexpr int kMxBias = 150;
 constexpr uint32_t kInfoExp = 0x1ffu, kInfoNaN = 1u << 9, kInfoInf = 1u << 10;
 
@@ -92,15 +96,16 @@ struct DecodePlan {
     size_t image_bytes;  // digit planes of one (pass, K chunk): kPlanes * cols * pitch * 16
 
     // ---- tcgen05 kernel (lq_gemv_tc.cu)
-    int tc_grid, tc_bpad, tc_n, tc_groups, tc_stages, tc_maxcontrib, tc_nq, tc_nacc, tc_nss, tc_nsa;
+    int tc_grid, tc_bpad, tc_n, tc_groups, tc_stages, tc_maxcontrib, tc_nq, tc_nacc, tc_nss, tc_nsa, tc_mt;
+    int tc_nqp, tc_kwp;     // pitches of the summaries (multiple of 4) and word deltas (of 16)
     long long tc_units;     // (row group, K stage) units over all groups
     size_t tc_smem;
     size_t row_bytes;       // bytes of one B row (one plane of one column): K / 2
 
     // ---- workspace (byte offsets from its 256-byte aligned base)
     //   mma.sync: hdr = ColHeader[batch], steps = StepSum[batch][nsteps], planes = images
-    //   tcgen05:  hdr = column summaries uint32 [batch][tc_nq], steps = binfo uint32
-    //             [batch][kw], planes = B rows [kMxPlanes * tc_bpad][K / 2] (row p * tc_bpad + c),
+    //   tcgen05:  hdr = column summaries uint32 [batch][tc_nqp], steps = word deltas
+    //             uint8 [batch][tc_kwp], planes = B rows [kMxPlanes * tc_bpad][K / 2] (row p * tc_bpad + c),
     //             count = group counters, slots = split partial sums
     size_t off_hdr, off_steps, off_planes, off_count, off_slots, bytes;
 };

@@ -240,6 +240,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     }
 
+    // lane 0 of the producer and issuer warps ran its role alone: reconverge
+    // every warp before the CTA barrier that orders the TMEM release
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -429,6 +432,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     }
 
+    // lane 0 of the producer and issuer warps ran its role alone: reconverge
+    // every warp before the CTA barrier that orders the TMEM release
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

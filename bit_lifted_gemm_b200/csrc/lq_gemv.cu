@@ -555,17 +555,20 @@ DecodePlan make_decode_plan(int out, int K, int batch) {
     pl.batch = batch;
     pl.nsteps = (pl.kw + kStepWords - 1) / kStepWords;
     pl.row_bytes = (size_t)pl.kw * 16;
-    // up to eight columns the mma.sync kernel is faster (measured); wider
-    // batches read the weights once on the tensor cores
-    pl.tc = batch > 8 && plan_tc(pl);
+    // Measured on B200 (13824 x 12288 and 28672 x 20480 layers): up to three
+    // columns the mma.sync kernel is faster, from four on the tensor-core
+    // kernel, which reads every weight once whatever the batch. Each takes the
+    // shapes the other cannot (the tensor-core kernel needs K a multiple of 256
+    // and at least 128 rows; the mma.sync kernel a word count its planes fit).
+    pl.tc = batch >= 4 && plan_tc(pl);
     if (!pl.tc && !plan_mma(pl) && !(pl.tc = plan_tc(pl))) return pl;
     size_t off = 0;
     if (pl.tc) {
         // column summaries, word info, digit planes, group counters, partial slots
         pl.off_hdr = off;
-        off = align256(off + (size_t)batch * pl.tc_nq * 4);
+        off = align256(off + (size_t)batch * pl.tc_nqp * 4);
         pl.off_steps = off;
-        off = align256(off + (size_t)batch * pl.kw * 4);
+        off = align256(off + (size_t)batch * pl.tc_kwp);
         pl.off_planes = off;
         off = align256(off + (size_t)pl.tc_n * pl.row_bytes);
         pl.off_count = off;

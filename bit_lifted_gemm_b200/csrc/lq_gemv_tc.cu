@@ -9,34 +9,39 @@
 //   * A = the signs as e2m1 +-1.0: a sign word becomes four 32-bit registers of
 //     eight nibbles (register r, nibble i <- bit r + 4i; one shift and one LOP3
 //     each), stored into tensor memory with tcgen05.st (one row per lane), so
-//     one M128 x K64 MMA consumes 8 KB of sign bits. Measured on B200: one such
-//     MMA per ~45.5 clocks per SM for N <= 64 -- 180 weight bits per clock, the
-//     rate at which HBM delivers them.
+//     one M128 x K64 MMA consumes 8 KB of sign bits.
 //   * B = the digit planes (row p * bpad + c: plane-major), TMA-loaded with the
 //     128-byte swizzle, in the element order of the sign expansion.
 //   * The scale of A is 1.0; the scale of B for row (p, c) and word w is
-//     2^(E_w - 1 - 3p - G_c): written per stage into tensor memory by the same
+//     2^(E_w - 1 - 3p - G_c): written per sub-stage into tensor memory by the
 //     warps that expand A (lane n % 32 of every quarter, column n / 32 of the
 //     MMA's four-column group), from the words' exponents and the column maxima
 //     G_c each CTA reduces from the quantizer's per-CTA summaries. Columns that
 //     hold +-Inf use scale 1.0 for plane 0 of their Inf words and 2^-127 for
 //     every other scale, so the accumulator holds (up to a negligible rest) the
 //     count of +Inf terms minus -Inf terms of each row; NaN columns output NaN.
+//   * Each M-tile has its own issuing warp. Measured on B200: a
+//     tcgen05.commit releases its mbarrier only ~400 clocks after the MMAs it
+//     covers, and one issuing thread's commits do not overlap, so a single
+//     issuer committing every four small MMAs runs the tensor pipe at a third of
+//     its rate; four issuers, each committing for its own tile, keep it busy.
 //
-// Work split: rows form groups of 256 (two M-tiles), K sub-stages of 8 words
-// (256 elements, four K64 MMAs). The (group, sub-stage) units in group-major
-// order are cut into one contiguous range per CTA, so every SM gets the same
-// number of MMAs whatever the shape. The sign words arrive by TMA in stages of
-// 32 words (128 bytes of each row, 128-byte swizzle), so DRAM serves whole
-// 128-byte runs of a row; each stage feeds up to four sub-stages. A CTA's run inside one group is a segment; its
-// accumulator is drained by the epilogue warps, which either store the result
-// (the segment covers the whole group) or write a float64 partial to a
-// workspace slot and count it in; the CTA that completes a group sums the
-// partials in slot order (deterministic) and stores.
-//   warp 0      TMA producer (weights, B, word info), one mbarrier ring
-//   warp 1      TMEM allocator and single-thread MMA issuer
-//   warps 2..5  sign expansion into TMEM A stages, B scale factors
-//   warps 6..9  column info, accumulator drain, partials, results
+// Work split: rows form groups of MT M-tiles of 128 (MT = 4 for narrow batches,
+// 2 for wide ones, whose accumulators take more tensor memory), K sub-stages
+// of 8 words (256 elements, four K64 MMAs per tile). The (group, sub-stage)
+// units in group-major order are cut into one contiguous range per CTA, so every
+// SM gets the same number of MMAs whatever the shape. The sign words arrive by
+// TMA in stages of 32 words (128 bytes of each row, 128-byte swizzle), so DRAM
+// serves whole 128-byte runs of a row; each stage feeds up to four sub-stages.
+// A CTA's run inside one group is a segment; its accumulators are drained by
+// the epilogue warps, which either store the result (the segment covers the
+// whole group) or write a float64 partial to a workspace slot and count it in;
+// the CTA that completes a group sums the partials in slot order
+// (deterministic) and stores.
+//   warp 0            TMA producer (weights, B, word info)
+//   warps 1..4        sign expansion into TMEM A slots, B scale factors
+//   warps 5..4+MT     one MMA issuer per M-tile (warp 5 also allocates TMEM)
+//   last four warps   column info, accumulator drain, partials, results
 // Every wait is bounded.
 #include <cuda.h>
 
@@ -52,46 +57,56 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kMT = 2;                              // M-tiles of 128 rows per group
-constexpr int kRG = 128 * kMT;                      // rows per group
-constexpr int kSub = 8;                             // words of K per sub-stage (4 MMAs of K64)
+constexpr int kSub = 8;                             // words of K per sub-stage (4 MMAs of K64 per tile)
 constexpr int kStageW = 32;                         // words of K per shared-memory stage (128 B per row)
-constexpr int kMaxSS = 6;                           // shared-memory stages (at most)
+constexpr int kMaxSS = 4;                           // shared-memory stages (at most)
 constexpr int kMaxSA = 4;                           // tensor-memory A / scale slots (at most)
-constexpr int kThreadsTc = 320;
 constexpr int kWTile = 128 * kStageW * 4;           // sign words of one M-tile in a stage: 16 KB
-constexpr int kACols = kMT * 32;                    // TMEM columns of an A slot
 constexpr int kSFCols = 16;                         // TMEM columns of a slot's B scales (4 per MMA)
 constexpr uint32_t kSpin = 1000000000u;             // bounded waits: 1 s
+
+constexpr int kExpWarps = 8;                        // sign expansion: two warps per TMEM lane quarter
+
+// warp 0 TMA, warps 1..8 expansion, MT issuers, four epilogue warps
+__host__ __device__ constexpr int tc_threads(int MT) { return 32 * (1 + kExpWarps + MT + 4); }
 
 struct TcArgs {
     const float* s;
     float* o;              // [batch][out]
-    const uint32_t* summ;  // [batch][nq] column summaries
+    const uint32_t* summ;  // [batch][nqp] quantizer summaries
     unsigned* count;       // [groups] arrivals per group (cleared by the quantizer)
-    double* slots;         // [groups][maxcontrib][batch][kRG]
+    double* slots;         // [groups][maxcontrib][batch][rows per group]
     unsigned* status;
     long long units;       // (group, sub-stage) units
-    int out, kw, batch, bpad, N, nq, groups, nsub, maxcontrib, nacc, nss, nsa;
+    int out, kw, batch, bpad, N, nq, nqp, groups, nsub, maxcontrib, nacc, nss, nsa;
 };
 
 struct Smem {
     size_t b, w, info, col, flag, bars, total;
-    size_t bstage, istage;
+    size_t bstage, istage, isumm;
 };
 
-__host__ __device__ inline Smem tc_smem(int N, int batch, int nss) {
+// Per stage: B (four sub-stage tiles of N rows x 128 B), the sign words of MT
+// tiles, and per column the 32 word deltas and the 4 quantizer summaries of
+// the stage (each region 128-byte aligned).
+__host__ __device__ inline Smem tc_smem(int MT, int N, int batch, int nss) {
     Smem L;
-    L.bstage = (size_t)4 * N * 128;                   // four sub-stage tiles of N rows x 128 B
-    L.istage = (size_t)batch * kStageW * 4;
+    L.bstage = (size_t)4 * N * 128;
+    L.isumm = ((size_t)batch * kStageW + 127) & ~(size_t)127;
+    L.istage = L.isumm + (((size_t)batch * 16 + 127) & ~(size_t)127);
     L.b = 0;
     L.w = L.b + nss * L.bstage;                        // multiples of 1024 (N is a multiple of 8)
-    L.info = L.w + (size_t)nss * kMT * kWTile;
-    L.col = L.info + ((nss * L.istage + 127) & ~(size_t)127);
+    L.info = L.w + (size_t)nss * MT * kWTile;
+    L.col = L.info + nss * L.istage;
     L.flag = L.col + 16 * 16;  // per column: G (biased), mode, Inf count
     L.bars = L.flag + 16;
-    L.total = L.bars + 8 * (3 * kMaxSS + 2 * kMaxSA + 4 + 1) + 1024 /*alignment slack*/;
+    L.total = L.bars + 8 * (3 * kMaxSS + 2 * kMaxSA + 4 + 4) + 1024 /*alignment slack*/;
     return L;
+}
+
+// Tensor-memory columns of the accumulators, A slots, B scale slots and A scales.
+__host__ __device__ inline int tc_tmem_cols(int MT, int N, int nacc, int nsa) {
+    return ((nacc * MT * N + 31) & ~31) + nsa * (MT * 32 + kSFCols) + 16;
 }
 
 // floor(i * n / parts) in 64-bit
@@ -123,6 +138,37 @@ __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&v)[16]) {
         : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
+// Sum the kMxPlanes plane columns (p * BP + c) of one accumulator tile into
+// part[c], c < BP: the tile's columns read 32 at a time.
+template <int BP, int C>
+__device__ __forceinline__ void drain_tile(uint32_t taddr, double (&part)[C]) {
+    static_assert(BP <= C, "plane columns beyond the partial sums");
+    constexpr int kCols = kMxPlanes * BP;
+    if constexpr (BP <= 4) {  // up to 28 columns: one load
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < kCols; ++e) part[e % BP] += (double)__uint_as_float(v[e]);
+    } else {  // 16 columns at a time (fewer live registers beside the 16 partial sums)
+#pragma unroll
+        for (int ch = 0; ch < (kCols + 15) / 16; ++ch) {
+            uint32_t v[16];
+            tmem_ld_x16(taddr + 16 * ch, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                if (16 * ch + e < kCols) part[(16 * ch + e) % BP] += (double)__uint_as_float(v[e]);
+        }
+    }
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]^T, kind::mxf4 with ue8m0 block scales of 32.
 __device__ __forceinline__ void umma_mxf4(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
                                           uint32_t sfb, uint32_t accumulate) {
@@ -131,10 +177,6 @@ __device__ __forceinline__ void umma_mxf4(uint32_t d, uint32_t a, uint64_t bdesc
         "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], [%1], %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
         "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
         : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d_(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
-    tma_load_3d(dst, map, x, y, z, bar);
 }
 
 // e2m1 +-1.0 nibbles of a sign word: register r, nibble i <- bit r + 4i.
@@ -152,7 +194,7 @@ __device__ __forceinline__ uint32_t idesc_mxf4(int N) {
     return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | (8u << 24);
 }
 
-// Walks a CTA's sub-stages: unit i -> (group, sub-stage), the index of its
+// Walks a CTA's sub-stages: unit -> (group, sub-stage), the index of its
 // shared-memory stage in the CTA's sequence (a new stage starts at every
 // 32-word boundary and at every group), and whether it is the last sub-stage
 // of that stage or of its group segment.
@@ -184,15 +226,23 @@ struct Walker {
     }
 };
 
-__global__ void __launch_bounds__(kThreadsTc, 1)
+template <int MT>
+__global__ void __launch_bounds__(tc_threads(MT), 1)
     gemv_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap bmap,
-                   const __grid_constant__ CUtensorMap imap, const TcArgs p) {
+                   const __grid_constant__ CUtensorMap dmap, const __grid_constant__ CUtensorMap smap,
+                   const TcArgs p) {
+    constexpr int kRG = 128 * MT;       // rows per group
+    constexpr int kACols = MT * 32;     // TMEM columns of an A slot
+    constexpr int kIss0 = 1 + kExpWarps;  // first issuer warp (it also owns the TMEM allocation)
+    constexpr int kEpi0 = kIss0 + MT;     // first epilogue warp
+    constexpr int kNamed1 = 32 * (kExpWarps + 4);  // expansion + epilogue warps
+    constexpr int kCmax = MT == 4 ? 4 : 16;        // batch columns (four M-tiles serve at most four)
     // the next kernel on the stream (the next layer's lift or quantizer) waits for
     // this grid before it reads anything; it may be scheduled as SMs free up
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    const Smem L = tc_smem(p.N, p.batch, p.nss);
+    const Smem L = tc_smem(MT, p.N, p.batch, p.nss);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nss = p.nss, nsa = p.nsa;
     int* col = reinterpret_cast<int*>(smem + L.col);        // [c][4]: biased G, mode, Inf count
@@ -209,24 +259,25 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         for (int st = 0; st < nss; ++st) {
             mbar_init(full_w + 8 * st, 1);
             mbar_init(full_b + 8 * st, 1);
-            mbar_init(freed + 8 * st, 4 + 1);  // four expansion warps read it, the MMAs consumed it
+            mbar_init(freed + 8 * st, kExpWarps + MT);  // the expansion warps read it, MT issuers consumed it
         }
         for (int a = 0; a < nsa; ++a) {
-            mbar_init(a_full + 8 * a, 4);
-            mbar_init(a_empty + 8 * a, 1);
+            mbar_init(a_full + 8 * a, kExpWarps);  // the expansion warps wrote every tile and the scales
+            mbar_init(a_empty + 8 * a, MT);      // every issuer's MMAs on it completed
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(acc_full + 8 * b, 1);
+            mbar_init(acc_full + 8 * b, MT);
             mbar_init(acc_empty + 8 * b, 4);
         }
-        mbar_init(done, 1);
+        for (int t = 0; t < MT; ++t) mbar_init(done + 8 * t, 1);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tensormap(&wmap);
         prefetch_tensormap(&bmap);
-        prefetch_tensormap(&imap);
+        prefetch_tensormap(&dmap);
+        prefetch_tensormap(&smap);
     }
-    if (warp == 1) {
+    if (warp == kIss0) {
         tmem_alloc(smem_addr(tmem_slot), 512);
         tmem_relinquish();
     }
@@ -234,8 +285,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // tensor-memory columns: accumulators, A slots, B scale slots, A scales
-    const uint32_t acol0 = (uint32_t)(p.nacc * kMT * p.N + 31) & ~31u;
+    const uint32_t acol0 = (uint32_t)(p.nacc * MT * p.N + 31) & ~31u;
     const uint32_t sfcol0 = acol0 + nsa * kACols, sfacol = sfcol0 + nsa * kSFCols;
 
     if (warp == 0) {
@@ -245,26 +295,26 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             wk.init(u0, u1, p.nsub);
             auto issue_w = [&](int ks, long long g, int stg) {
                 const int slot = ks % nss;
-                mbar_arrive_expect_tx(full_w + 8 * slot, kMT * kWTile);
-                for (int t = 0; t < kMT; ++t)
-                    tma_load_2d(smem_addr(smem + L.w + ((size_t)slot * kMT + t) * kWTile), &wmap, stg * kStageW,
+                mbar_arrive_expect_tx(full_w + 8 * slot, MT * kWTile);
+                for (int t = 0; t < MT; ++t)
+                    tma_load_2d(smem_addr(smem + L.w + ((size_t)slot * MT + t) * kWTile), &wmap, stg * kStageW,
                                 (int)(g * kRG) + 128 * t, full_w + 8 * slot);
             };
             auto issue_b = [&](int ks, int stg) {
                 const int slot = ks % nss;
-                mbar_arrive_expect_tx(full_b + 8 * slot, (uint32_t)(L.bstage + L.istage));
-                tma_load_3d_(smem_addr(smem + L.b + slot * L.bstage), &bmap, 0, 0, stg * 4, full_b + 8 * slot);
-                tma_load_2d(smem_addr(smem + L.info + slot * L.istage), &imap, stg * kStageW, 0, full_b + 8 * slot);
+                const uint32_t ib = smem_addr(smem + L.info + slot * L.istage);
+                mbar_arrive_expect_tx(full_b + 8 * slot, (uint32_t)(L.bstage + p.batch * (kStageW + 16)));
+                tma_load_3d(smem_addr(smem + L.b + slot * L.bstage), &bmap, 0, 0, stg * 4, full_b + 8 * slot);
+                tma_load_2d(ib, &dmap, stg * kStageW, 0, full_b + 8 * slot);
+                tma_load_2d(ib + (uint32_t)L.isumm, &smap, stg * 4, 0, full_b + 8 * slot);
             };
-            // stage list of this CTA: (group, 32-word stage) in order
             // the sign words do not depend on the kernel before this one: request
             // the first stages before waiting for it
             int early = 0;
             {
                 Walker e = wk;
                 for (long long u = u0; u < u1 && early < nss; ++u) {
-                    const bool sl = e.stage_last(u);
-                    if (sl) {
+                    if (e.stage_last(u)) {
                         issue_w(early, e.g, e.sub >> 2);
                         ++early;
                     }
@@ -295,8 +345,106 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 if (ks < issued) mbar_wait(full_b + 8 * (ks % nss), (ks / nss) & 1, p.status, kSpin);
             }
         }
-    } else if (warp == 1) {
-        // ================================================================ MMA issuer
+    } else if (warp <= kExpWarps) {
+        // ================================================================ sign expansion, B scales
+        // Each lane quarter's 32 rows of the MT tiles are split between its two
+        // warps k: warp k expands tiles k MT/2 .. (k+1) MT/2 - 1 and writes the B
+        // scales of MMAs kk = 2k, 2k + 1 (words 4k .. 4k + 3 of the sub-stage).
+        // More warps do not help: the tensor-memory stores of the expanded
+        // operand (four bytes per sign byte) set the pace.
+        const int q = warp & 3;                 // TMEM lane quarter of this warp
+        const int k = (warp - 1) >> 2;          // 0..1
+        const int r = 32 * q + lane;            // row within each M-tile
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        if (k == 0) {  // A scales: 1.0 for every row and block
+            uint32_t one[16];
+#pragma unroll
+            for (int x = 0; x < 16; ++x) one[x] = 0x7F7F7F7Fu;
+            tmem_st_x16(lane_base + sfacol, one);
+        }
+        named_bar(1, kNamed1);  // column info from the epilogue warps
+        // this lane's B rows n = 32 c4 + lane: column, scale base 126 - 3p - G_c (biased), mode
+        // (four M-tiles serve at most four columns: 28 B rows, one block of 32)
+        constexpr int kRB = MT == 4 ? 1 : 4;
+        int rc[kRB], rbase[kRB], rmode[kRB];
+        bool rp0[kRB];
+#pragma unroll
+        for (int c4 = 0; c4 < kRB; ++c4) {
+            const int n = 32 * c4 + lane;
+            const int pl = n / p.bpad, c = n - pl * p.bpad;
+            const bool live = n < p.N && pl < kMxPlanes && c < p.batch;
+            rc[c4] = live ? c : 0;
+            rmode[c4] = live ? col[4 * c + 1] : -1;
+            rbase[c4] = live ? 126 - 3 * pl - col[4 * c] : 0;
+            rp0[c4] = pl == 0;
+        }
+        const int nrows4 = (p.N + 31) / 32;  // row blocks of 32 that hold B rows
+        Walker wk;
+        wk.init(u0, u1, p.nsub);
+        int i = 0;
+        for (long long u = u0; u < u1; ++u, ++i) {
+            const int ks = wk.ks, slot = ks % nss, j = wk.sub & 3, a = i % nsa;
+            bool ok = mbar_wait(full_w + 8 * slot, (ks / nss) & 1, p.status, kSpin);
+            ok = ok && mbar_wait(full_b + 8 * slot, (ks / nss) & 1, p.status, kSpin);
+            ok = ok && (i < nsa || mbar_wait(a_empty + 8 * a, ((i / nsa) - 1) & 1, p.status, kSpin));
+            if (!__all_sync(0xffffffffu, ok) || *abort_flag) {  // tcgen05.st is warp-collective
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            // ---- A: the 8 words of row r of this warp's tiles (128-byte swizzle:
+            // 16-byte chunk c at c ^ (r & 7))
+#pragma unroll
+            for (int tt = 0; tt < MT / 2; ++tt) {
+                const int t = k * (MT / 2) + tt;
+                const uint8_t* row = smem + L.w + ((size_t)slot * MT + t) * kWTile + (size_t)r * 128;
+                const uint4 w0 = *reinterpret_cast<const uint4*>(row + (((2 * j) ^ (r & 7)) << 4));
+                const uint4 w1 = *reinterpret_cast<const uint4*>(row + (((2 * j + 1) ^ (r & 7)) << 4));
+                uint32_t v[32];
+                expand_word(w0.x, v);
+                expand_word(w0.y, v + 4);
+                expand_word(w0.z, v + 8);
+                expand_word(w0.w, v + 12);
+                expand_word(w1.x, v + 16);
+                expand_word(w1.y, v + 20);
+                expand_word(w1.z, v + 24);
+                expand_word(w1.w, v + 28);
+                tmem_st_32x32b_x32(lane_base + acol0 + a * kACols + t * 32, v);
+            }
+            // ---- B scales of MMAs kk = 2k, 2k + 1: words 8 j + 4k .. + 3 of each live
+            // row's column; scale column 4 kk + c4, bytes 0 and 1 for the MMA's two
+            // blocks of 32
+            const uint8_t* dsm = smem + L.info + slot * L.istage;
+            const uint32_t* ssm = reinterpret_cast<const uint32_t*>(dsm + L.isumm);
+            uint32_t sf[8] = {0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu,
+                              0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu};
+#pragma unroll
+            for (int c4 = 0; c4 < kRB; ++c4) {
+                uint32_t e4 = 0x7F7F7F7Fu;  // rows without a B row: any finite scale
+                if (c4 < nrows4 && rmode[c4] >= 0) {
+                    const uint32_t dl = *reinterpret_cast<const uint32_t*>(dsm + rc[c4] * kStageW + 8 * j + 4 * k);
+                    if (rmode[c4] == kColFinite) {
+                        // 2^(E - 1 - 3p - G_c): base 126 - 3p - (G_c - E_loc), less each word's delta
+                        const int base = max(0, rbase[c4] + (int)(ssm[4 * rc[c4] + j] & kInfoExp));
+                        e4 = __vsubus4((uint32_t)base * 0x01010101u, dl & 0x7F7F7F7Fu);
+                    } else if (rmode[c4] == kColInf) {
+                        e4 = rp0[c4] ? ((dl >> 7) & 0x01010101u) * 127u : 0u;  // plane 0 of Inf words: 1.0
+                    }
+                }
+                sf[c4] = __byte_perm(e4, 0x7F7F7F7Fu, 0x4410);      // words 0, 1 of the four: MMA kk = 2k
+                sf[4 + c4] = __byte_perm(e4, 0x7F7F7F7Fu, 0x4432);  // words 2, 3: MMA kk = 2k + 1
+            }
+            tmem_st_x8(lane_base + sfcol0 + a * kSFCols + 8 * k, sf);
+            __syncwarp();
+            if (lane == 0 && wk.stage_last(u)) mbar_arrive(freed + 8 * slot);  // read all it needs from the stage
+            tmem_st_wait();
+            tc_fence_before();
+            if (lane == 0) mbar_arrive(a_full + 8 * a);
+            wk.next(u);
+        }
+    } else if (warp < kEpi0) {
+        // ================================================================ MMA issuer of M-tile t
+        const int t = warp - kIss0;
         if (lane == 0) {
             const uint32_t idesc = idesc_mxf4(p.N);
             int buf = 0;
@@ -317,16 +465,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 }
                 tc_fence_after();
                 const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + L.b + slot * L.bstage + (size_t)j * p.N * 128));
-                const uint32_t acc = tmem + (uint32_t)(buf * kMT * p.N);
+                const uint32_t acc = tmem + (uint32_t)((buf * MT + t) * p.N);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-                    for (int t = 0; t < kMT; ++t)
-                        umma_mxf4(acc + t * p.N, tmem + acol0 + a * kACols + t * 32 + kk * 8,
-                                  bdesc + (uint64_t)((kk * 32) >> 4), idesc, tmem + sfacol,
-                                  tmem + sfcol0 + a * kSFCols + 4 * kk, (uint32_t)(!first || kk > 0));
-                if (wk.stage_last(u)) umma_commit(freed + 8 * slot);
+                    umma_mxf4(acc, tmem + acol0 + a * kACols + t * 32 + kk * 8, bdesc + (uint64_t)((kk * 32) >> 4),
+                              idesc, tmem + sfacol, tmem + sfcol0 + a * kSFCols + 4 * kk, (uint32_t)(!first || kk > 0));
                 umma_commit(a_empty + 8 * a);
+                if (wk.stage_last(u)) umma_commit(freed + 8 * slot);
                 if (last) {
                     umma_commit(acc_full + 8 * buf);
                     ++uses[buf];
@@ -334,115 +479,19 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 }
                 wk.next(u);
             }
-            umma_commit(done);  // fires when every MMA issued above has completed
-            mbar_wait(done, 0, p.status, kSpin);
-        }
-    } else if (warp < 6) {
-        // ================================================================ sign expansion, B scales
-        const int q = warp & 3;  // TMEM lane quarter of this warp
-        const int r = 32 * q + lane;  // row within each M-tile
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-        {   // A scales: 1.0 for every row and block
-            uint32_t one[16];
-#pragma unroll
-            for (int x = 0; x < 16; ++x) one[x] = 0x7F7F7F7Fu;
-            tmem_st_x16(lane_base + sfacol, one);
-        }
-        named_bar(1, 256);  // column info from the epilogue warps
-        // this lane's B rows n = 32 c4 + lane: column, plane, exponent offset, mode
-        int rc[4], rbase[4], rmode[4];
-        bool rinf0[4];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            const int n = 32 * c4 + lane;
-            const int pl = n / p.bpad, c = n - pl * p.bpad;
-            const bool live = n < p.N && pl < kMxPlanes && c < p.batch;
-            rc[c4] = live ? c : 0;
-            rmode[c4] = live ? col[4 * c + 1] : -1;
-            rbase[c4] = live ? 126 - 3 * pl - col[4 * c] : 0;
-            rinf0[c4] = pl == 0;
-        }
-        const int nrows4 = (p.N + 31) / 32;  // row blocks of 32 that hold B rows
-        Walker wk;
-        wk.init(u0, u1, p.nsub);
-        int i = 0;
-        for (long long u = u0; u < u1; ++u, ++i) {
-            const int ks = wk.ks, slot = ks % nss, j = wk.sub & 3, a = i % nsa;
-            bool ok = mbar_wait(full_w + 8 * slot, (ks / nss) & 1, p.status, kSpin);
-            ok = ok && mbar_wait(full_b + 8 * slot, (ks / nss) & 1, p.status, kSpin);
-            ok = ok && (i < nsa || mbar_wait(a_empty + 8 * a, ((i / nsa) - 1) & 1, p.status, kSpin));
-            if (!__all_sync(0xffffffffu, ok) || *abort_flag) {  // tcgen05.st is warp-collective
-                *abort_flag = 1;
-                break;
-            }
-            tc_fence_after();
-            // ---- A: 8 words of row r of each M-tile (128-byte swizzle: chunk c at c ^ (r & 7))
-#pragma unroll
-            for (int t = 0; t < kMT; ++t) {
-                const uint8_t* row = smem + L.w + ((size_t)slot * kMT + t) * kWTile + (size_t)r * 128;
-                const uint4 w0 = *reinterpret_cast<const uint4*>(row + (((2 * j) ^ (r & 7)) << 4));
-                const uint4 w1 = *reinterpret_cast<const uint4*>(row + (((2 * j + 1) ^ (r & 7)) << 4));
-                uint32_t v[32];
-                expand_word(w0.x, v);
-                expand_word(w0.y, v + 4);
-                expand_word(w0.z, v + 8);
-                expand_word(w0.w, v + 12);
-                expand_word(w1.x, v + 16);
-                expand_word(w1.y, v + 20);
-                expand_word(w1.z, v + 24);
-                expand_word(w1.w, v + 28);
-                tmem_st_32x32b_x32(lane_base + acol0 + a * kACols + t * 32, v);
-            }
-            // ---- B scales of the sub-stage: word 8 j + 2 kk + h of each live row's column
-            const uint32_t* info = reinterpret_cast<const uint32_t*>(smem + L.info + slot * L.istage);
-            uint32_t sf[16];
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                if (c4 >= nrows4 || rmode[c4] < 0) {  // no B row here: any finite scale
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) sf[4 * kk + c4] = 0x7F7F7F7Fu;
-                    continue;
-                }
-                const uint4 ia = *reinterpret_cast<const uint4*>(info + rc[c4] * kStageW + 8 * j);
-                const uint4 ib = *reinterpret_cast<const uint4*>(info + rc[c4] * kStageW + 8 * j + 4);
-                const uint32_t iw[8] = {ia.x, ia.y, ia.z, ia.w, ib.x, ib.y, ib.z, ib.w};
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    uint32_t bytes = 0x7F7F0000u;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint32_t x = iw[2 * kk + h];
-                        const int eb = (int)(x & kInfoExp);
-                        int e;
-                        if (rmode[c4] == kColFinite)
-                            e = eb == 0 ? 0 : min(254, max(0, eb + rbase[c4]));
-                        else if (rmode[c4] == kColInf)
-                            e = (rinf0[c4] && (x & kInfoInf)) ? 127 : 0;
-                        else
-                            e = 127;
-                        bytes |= (uint32_t)e << (8 * h);
-                    }
-                    sf[4 * kk + c4] = bytes;
-                }
-            }
-            tmem_st_x16(lane_base + sfcol0 + a * kSFCols, sf);
-            __syncwarp();
-            if (lane == 0 && wk.stage_last(u)) mbar_arrive(freed + 8 * slot);  // read all it needs from the stage
-            tmem_st_wait();
-            tc_fence_before();
-            if (lane == 0) mbar_arrive(a_full + 8 * a);
-            wk.next(u);
+            umma_commit(done + 8 * t);  // fires when every MMA issued above has completed
+            mbar_wait(done + 8 * t, 0, p.status, kSpin);
         }
     } else {
         // ================================================================ column info, drain, results
         const int q = warp & 3;
-        const int et = threadIdx.x - 192;  // 0..127
+        const int et = threadIdx.x - 32 * kEpi0;  // 0..127
         asm volatile("griddepcontrol.wait;" ::: "memory");
         // column info: biased max exponent, mode, Inf count, from the per-CTA summaries
-        for (int c = warp - 6; c < p.batch; c += 4) {
+        for (int c = warp - kEpi0; c < p.batch; c += 4) {
             uint32_t e = 0, f = 0, n = 0;
             for (int jj = lane; jj < p.nq; jj += 32) {
-                const uint32_t v = p.summ[(size_t)c * p.nq + jj];
+                const uint32_t v = p.summ[(size_t)c * p.nqp + jj];
                 e = max(e, v & kInfoExp);
                 f |= v & (kInfoNaN | kInfoInf);
                 n += v >> 16;
@@ -456,7 +505,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 col[4 * c + 2] = (int)n;
             }
         }
-        named_bar(1, 256);
+        named_bar(1, kNamed1);
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L.flag + 8);
         int buf = 0, use[2] = {0, 0};
@@ -476,20 +525,60 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             named_bar(2, 128);
             if (*last_flag) break;
             tc_fence_after();
-            // ---- drain: per M-tile, sum the planes of each column (plane p = columns p * bpad ..)
-            double part[kMT][16];
+            double* slot = p.slots + ((size_t)(g * p.maxcontrib + jslot) * p.batch) * kRG;
+            // store the results of tile t of group g from the plane sums x[c]
+            auto store_tile = [&](int t, const double (&x)[kCmax]) {
+                const long long r = g * kRG + t * 128 + 32 * q + lane;
+                if (r >= p.out) return;
+                const double sr = (double)__ldg(p.s + r);
 #pragma unroll
-            for (int t = 0; t < kMT; ++t) {
-#pragma unroll
-                for (int c = 0; c < 16; ++c) part[t][c] = 0.0;
+                for (int c = 0; c < kCmax; ++c) {
+                    if (c >= p.batch) continue;
+                    const int mode = col[4 * c + 1];
+                    float res;
+                    if (mode == kColFinite) {
+                        // undo the column normalization 2^-G_c (G_c = biased - kMxBias)
+                        const double scale = __longlong_as_double((long long)(col[4 * c] - kMxBias + 1023) << 52);
+                        res = (float)(x[c] * scale * sr);
+                    } else if (mode == kColInf) {
+                        const double S = rint(x[c]);
+                        const double n = (double)col[4 * c + 2];
+                        const double inf = __longlong_as_double(0x7ff0000000000000ll);
+                        const double val = S == n ? inf : S == -n ? -inf : __longlong_as_double(0x7ff8000000000000ll);
+                        res = (float)(val * sr);
+                    } else {
+                        res = __int_as_float(0x7fc00000);
+                    }
+                    p.o[(size_t)c * p.out + r] = res;
+                }
+            };
+            // ---- drain tile by tile: sum the planes of each column (plane p =
+            // columns p * bpad ..), then store the result (the group is this
+            // CTA's alone) or the partial to slot (g, jslot)
 #pragma unroll 1
-                for (int pl = 0; pl < kMxPlanes; ++pl) {
-                    uint32_t v[16];
-                    tmem_ld_x16(lane_base + (uint32_t)(buf * kMT * p.N + t * p.N + pl * p.bpad), v);
-                    tmem_ld_wait();
+            for (int t = 0; t < MT; ++t) {
+                double part[kCmax];
 #pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        if (c < p.bpad) part[t][c] += (double)__uint_as_float(v[c]);
+                for (int c = 0; c < kCmax; ++c) part[c] = 0.0;
+                const uint32_t tacc = lane_base + (uint32_t)((buf * MT + t) * p.N);
+                if (p.bpad == 1) {
+                    drain_tile<1>(tacc, part);
+                } else if (p.bpad == 2) {
+                    drain_tile<2>(tacc, part);
+                } else if (p.bpad == 4 || MT == 4) {
+                    drain_tile<4>(tacc, part);
+                } else if constexpr (MT == 2) {
+                    if (p.bpad == 8)
+                        drain_tile<8>(tacc, part);
+                    else
+                        drain_tile<16>(tacc, part);
+                }
+                if (nc == 1) {
+                    store_tile(t, part);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < kCmax; ++c)
+                        if (c < p.batch) slot[(size_t)c * kRG + t * 128 + 32 * q + lane] = part[c];
                 }
             }
             tc_fence_before();
@@ -497,15 +586,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             ++use[buf];
             buf = p.nacc == 2 ? buf ^ 1 : 0;
 
-            bool final_here = nc == 1;
-            if (!final_here) {
-                // partial to slot (g, jslot); the CTA that completes group g sums them
-                double* slot = p.slots + ((size_t)(g * p.maxcontrib + jslot) * p.batch) * kRG;
-#pragma unroll
-                for (int t = 0; t < kMT; ++t)
-#pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        if (c < p.batch) slot[(size_t)c * kRG + t * 128 + 32 * q + lane] = part[t][c];
+            if (nc > 1) {
+                // the CTA that completes group g sums the partials in slot order
                 __threadfence();
                 named_bar(2, 128);
                 if (et == 0) {
@@ -515,47 +597,20 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                     *last_flag = last;
                 }
                 named_bar(2, 128);
-                final_here = *last_flag != 0;
-                if (final_here) {
+                if (*last_flag != 0) {
                     __threadfence();
                     const double* base = p.slots + ((size_t)(g * p.maxcontrib) * p.batch) * kRG;
+#pragma unroll 1
+                    for (int t = 0; t < MT; ++t) {
+                        double sum[kCmax];
 #pragma unroll
-                    for (int t = 0; t < kMT; ++t)
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
+                        for (int c = 0; c < kCmax; ++c) {
+                            sum[c] = 0.0;
                             if (c >= p.batch) continue;
-                            double sum = 0.0;
                             for (int jj = 0; jj < nc; ++jj)
-                                sum += __ldcg(base + ((size_t)jj * p.batch + c) * kRG + t * 128 + 32 * q + lane);
-                            part[t][c] = sum;
+                                sum[c] += __ldcg(base + ((size_t)jj * p.batch + c) * kRG + t * 128 + 32 * q + lane);
                         }
-                }
-            }
-            if (final_here) {
-#pragma unroll
-                for (int t = 0; t < kMT; ++t) {
-                    const long long r = g * kRG + t * 128 + 32 * q + lane;
-                    if (r >= p.out) continue;
-                    const double sr = (double)__ldg(p.s + r);
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        if (c >= p.batch) continue;
-                        const int mode = col[4 * c + 1];
-                        float res;
-                        if (mode == kColFinite) {
-                            // undo the column normalization 2^-G_c (G_c = biased - kMxBias)
-                            const double scale = __longlong_as_double((long long)(col[4 * c] - kMxBias + 1023) << 52);
-                            res = (float)(part[t][c] * scale * sr);
-                        } else if (mode == kColInf) {
-                            const double S = rint(part[t][c]);
-                            const double n = (double)col[4 * c + 2];
-                            const double inf = __longlong_as_double(0x7ff0000000000000ll);
-                            const double val = S == n ? inf : S == -n ? -inf : __longlong_as_double(0x7ff8000000000000ll);
-                            res = (float)(val * sr);
-                        } else {
-                            res = __int_as_float(0x7fc00000);
-                        }
-                        p.o[(size_t)c * p.out + r] = res;
+                        store_tile(t, sum);
                     }
                 }
             }
@@ -563,9 +618,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
     }
 
+    // lane 0 of several warps ran its role alone: reconverge every warp before
+    // the CTA barrier that orders the TMEM release after all tensor-memory use
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kIss0) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -606,33 +664,36 @@ bool plan_tc(DecodePlan& p) {
     while (bpad < p.batch) bpad *= 2;
     p.tc_bpad = bpad;
     p.tc_n = (kMxPlanes * bpad + 7) / 8 * 8;
-    p.tc_groups = (p.out + kRG - 1) / kRG;
+    // tiles per group (four issuers when the accumulators allow), A / scale slots
+    // (at least two), accumulator buffers: the first that fits tensor memory
+    p.tc_mt = 0;
+    for (int mt = bpad <= 4 ? 4 : 2; mt >= 2 && !p.tc_mt; mt -= 2)
+        for (int nsa = kMaxSA; nsa >= 2 && !p.tc_mt; --nsa)
+            for (int nacc = 2; nacc >= 1; --nacc)
+                if (tc_tmem_cols(mt, p.tc_n, nacc, nsa) <= 512) {
+                    p.tc_mt = mt;
+                    p.tc_nsa = nsa;
+                    p.tc_nacc = nacc;
+                    break;
+                }
+    if (!p.tc_mt) return false;
+    const int rg = 128 * p.tc_mt;
+    p.tc_groups = (p.out + rg - 1) / rg;
     p.tc_stages = (p.kw + kSub - 1) / kSub;  // sub-stages per group
     p.tc_units = (long long)p.tc_groups * p.tc_stages;
     p.tc_grid = (int)std::min<long long>(sm_count(), p.tc_units);
     p.tc_nq = (p.kw + kMxQWords - 1) / kMxQWords;
-    // tensor memory: accumulators (double-buffered when they fit), A and scale slots
-    p.tc_nacc = 0;
-    p.tc_nsa = 0;
-    for (int nsa = kMaxSA; nsa >= 2 && !p.tc_nacc; --nsa)
-        for (int nacc = 2; nacc >= 1; --nacc) {
-            const int acc = (nacc * kMT * p.tc_n + 31) & ~31;
-            if (acc + nsa * (kACols + kSFCols) + 16 <= 512) {
-                p.tc_nacc = nacc;
-                p.tc_nsa = nsa;
-                break;
-            }
-        }
-    if (!p.tc_nacc) return false;
+    p.tc_nqp = (p.tc_nq + 3) & ~3;   // 16-byte rows for the summary copies
+    p.tc_kwp = (p.kw + 15) & ~15;    // 16-byte rows for the delta copies
     // shared memory: as many stages as fit, up to kMaxSS
     p.tc_nss = 0;
     for (int nss = kMaxSS; nss >= 2; --nss)
-        if (tc_smem(p.tc_n, p.batch, nss).total <= 227 * 1024) {
+        if (tc_smem(p.tc_mt, p.tc_n, p.batch, nss).total <= 227 * 1024) {
             p.tc_nss = nss;
             break;
         }
     if (!p.tc_nss) return false;
-    p.tc_smem = tc_smem(p.tc_n, p.batch, p.tc_nss).total;
+    p.tc_smem = tc_smem(p.tc_mt, p.tc_n, p.batch, p.tc_nss).total;
     // most CTAs that share one group
     auto cta_of_h = [&](long long x) {
         long long b = x * p.tc_grid / p.tc_units;
@@ -650,14 +711,14 @@ bool plan_tc(DecodePlan& p) {
 }
 
 size_t tc_slot_bytes(const DecodePlan& p) {
-    return p.tc_maxcontrib > 1 ? (size_t)p.tc_groups * p.tc_maxcontrib * p.batch * kRG * sizeof(double) : 0;
+    return p.tc_maxcontrib > 1 ? (size_t)p.tc_groups * p.tc_maxcontrib * p.batch * (128 * p.tc_mt) * sizeof(double) : 0;
 }
 
 cudaError_t launch_gemv_tc(const uint32_t* packed, const float* s, const DecodePlan& pl, float* o, uint8_t* ws,
                            unsigned* status, cudaStream_t st) {
     EncodeTiledFn encode = encode_fn_tc();
     if (!encode) return cudaErrorNotSupported;
-    CUtensorMap wmap, bmap, imap;
+    CUtensorMap wmap, bmap, dmap, smap;
     {  // sign words [out][kw], box 32 words (128 B) x 128 rows, 128-byte swizzle
         cuuint64_t gdim[2] = {(cuuint64_t)pl.kw, (cuuint64_t)pl.out};
         cuuint64_t gstride[1] = {(cuuint64_t)pl.kw * 4};
@@ -679,12 +740,22 @@ cudaError_t launch_gemv_tc(const uint32_t* packed, const float* s, const DecodeP
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    {  // word info [batch][kw], box 32 words x batch
-        cuuint64_t gdim[2] = {(cuuint64_t)pl.kw, (cuuint64_t)pl.batch};
-        cuuint64_t gstride[1] = {(cuuint64_t)pl.kw * 4};
+    {  // word deltas [batch][kwp] bytes, box 32 words x batch
+        cuuint64_t gdim[2] = {(cuuint64_t)pl.tc_kwp, (cuuint64_t)pl.batch};
+        cuuint64_t gstride[1] = {(cuuint64_t)pl.tc_kwp};
         cuuint32_t box[2] = {kStageW, (cuuint32_t)pl.batch};
         cuuint32_t es[2] = {1, 1};
-        if (encode(&imap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, ws + pl.off_steps, gdim, gstride, box, es,
+        if (encode(&dmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ws + pl.off_steps, gdim, gstride, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {  // quantizer summaries [batch][nqp], box 4 (the sub-stages of a stage) x batch
+        cuuint64_t gdim[2] = {(cuuint64_t)pl.tc_nqp, (cuuint64_t)pl.batch};
+        cuuint64_t gstride[1] = {(cuuint64_t)pl.tc_nqp * 4};
+        cuuint32_t box[2] = {4, (cuuint32_t)pl.batch};
+        cuuint32_t es[2] = {1, 1};
+        if (encode(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, ws + pl.off_hdr, gdim, gstride, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
@@ -703,6 +774,7 @@ cudaError_t launch_gemv_tc(const uint32_t* packed, const float* s, const DecodeP
     a.bpad = pl.tc_bpad;
     a.N = pl.tc_n;
     a.nq = pl.tc_nq;
+    a.nqp = pl.tc_nqp;
     a.groups = pl.tc_groups;
     a.nsub = pl.tc_stages;
     a.maxcontrib = pl.tc_maxcontrib;
@@ -710,17 +782,19 @@ cudaError_t launch_gemv_tc(const uint32_t* packed, const float* s, const DecodeP
     a.nss = pl.tc_nss;
     a.nsa = pl.tc_nsa;
 
-    static size_t granted[64] = {};
+    auto kern = pl.tc_mt == 4 ? gemv_tc_kernel<4> : gemv_tc_kernel<2>;
+    static size_t granted[2][64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 64 || granted[dev] < pl.tc_smem) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.tc_smem);
+    const int ki = pl.tc_mt == 4 ? 1 : 0;
+    if (dev >= 64 || granted[ki][dev] < pl.tc_smem) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.tc_smem);
         if (e != cudaSuccess) return e;
-        if (dev < 64) granted[dev] = pl.tc_smem;
+        if (dev < 64) granted[ki][dev] = pl.tc_smem;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.tc_grid, 1, 1);
-    cfg.blockDim = dim3(kThreadsTc, 1, 1);
+    cfg.blockDim = dim3(tc_threads(pl.tc_mt), 1, 1);
     cfg.dynamicSmemBytes = pl.tc_smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -728,7 +802,7 @@ cudaError_t launch_gemv_tc(const uint32_t* packed, const float* s, const DecodeP
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemv_tc_kernel, wmap, bmap, imap, a);
+    return cudaLaunchKernelEx(&cfg, kern, wmap, bmap, dmap, smap, a);
 }
 
 }  // namespace lq

@@ -462,6 +462,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
             }
         }
     }
+    __syncwarp();  // reconverge the producer and issuer warps before the CTA barrier
     __syncthreads();
     if (done && !*abort_flag) {
         const int tid = threadIdx.x, w = tid - 64;  // the generic forms use warps 2..9
@@ -490,6 +491,9 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
         }
     }
 
+    // lane 0 of the producer and issuer warps ran its role alone: reconverge
+    // every warp before the CTA barrier that orders the TMEM release
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

@@ -159,10 +159,10 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const QuantArgs a) 
 struct QuantMxArgs {
     const float* u;
     uint8_t* planes;   // [kMxPlanes * bpad][K / 2]: row p * bpad + c
-    uint32_t* binfo;   // [batch][kw]
-    uint32_t* summ;    // [batch][nq]
+    uint8_t* delta;    // [batch][kwp]: per word, its exponent below the CTA's largest (and an Inf flag)
+    uint32_t* summ;    // [batch][nqp]: per quantizer CTA
     unsigned* zero;    // group counters of the contraction, cleared here
-    int K, kw, bpad, nq, nzero;
+    int K, kw, kwp, bpad, nq, nqp, nzero;
 };
 
 __global__ void __launch_bounds__(32 * kMxQWords) quant_mx_kernel(const QuantMxArgs a) {
@@ -229,12 +229,15 @@ __global__ void __launch_bounds__(32 * kMxQWords) quant_mx_kernel(const QuantMxA
             v |= __shfl_xor_sync(0xffffffffu, v, 16);
             if (lane < 4) *reinterpret_cast<uint32_t*>(dst + (size_t)(p * a.bpad + c) * (a.K / 2)) = v;
         }
-        if (lane == 0) a.binfo[(size_t)c * a.kw + w] = info;
         summ = (info & (kInfoNaN | kInfoInf)) ? (info & (kInfoNaN | kInfoInf)) | (ninf << 16) : info;
     }
     if (lane == 0) s_sum[warp] = summ;
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (lane == 0) {
+        // the CTA's largest exponent over its finite words; each word stores how
+        // far below it its own exponent lies (at most 127: further down, its
+        // scales underflow to the smallest ue8m0 value whatever the column),
+        // bit 7 marking a word that holds +-Inf; all-zero and NaN words store 127
         uint32_t e = 0, f = 0, n = 0;
         for (int i = 0; i < kMxQWords; ++i) {
             const uint32_t v = s_sum[i];
@@ -242,7 +245,16 @@ __global__ void __launch_bounds__(32 * kMxQWords) quant_mx_kernel(const QuantMxA
             f |= v & (kInfoNaN | kInfoInf);
             n += v >> 16;
         }
-        a.summ[(size_t)c * a.nq + blockIdx.x] = e | f | (n << 16);
+        if (w < a.kw) {
+            const uint32_t v = s_sum[warp];
+            uint32_t db = 0x7Fu;
+            if (v & kInfoInf)
+                db = 0xFFu;
+            else if (!(v & kInfoNaN) && (v & kInfoExp) != 0u)
+                db = min(127u, e - (v & kInfoExp));
+            a.delta[(size_t)c * a.kwp + w] = (uint8_t)db;
+        }
+        if (warp == 0) a.summ[(size_t)c * a.nqp + blockIdx.x] = e | f | (n << 16);
     }
 }
 
@@ -253,13 +265,15 @@ cudaError_t launch_quant_mx(const float* u, const DecodePlan& p, void* ws, cudaS
     QuantMxArgs a;
     a.u = u;
     a.planes = w + p.off_planes;
-    a.binfo = reinterpret_cast<uint32_t*>(w + p.off_steps);
+    a.delta = w + p.off_steps;
     a.summ = reinterpret_cast<uint32_t*>(w + p.off_hdr);
     a.zero = reinterpret_cast<unsigned*>(w + p.off_count);
     a.K = p.K;
     a.kw = p.kw;
     a.bpad = p.tc_bpad;
     a.nq = p.tc_nq;
+    a.nqp = p.tc_nqp;
+    a.kwp = p.tc_kwp;
     a.nzero = p.tc_groups;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.tc_nq, p.batch, 1);
