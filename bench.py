@@ -51,11 +51,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 METRIC = "decode GEMV packed-weight GB/s (% of HBM) and prefill TFLOP/s, per LQ-D/d"
 
 
-def workload_config(cfg, name, world):
+def workload_config(cfg, name, world, shard=False):
     return {"workload": name, "in": cfg.in_dim, "out": cfg.out, "d": cfg.d, "D": cfg.D, "K": cfg.K,
-            "batch": 1, "tblk": cfg.tblk, "step": "lq_lift_gemv (lift + gemv)", "parallelism": f"replicas{world}",
-            "arith": "lift fp32; u as 32-bit fixed point in four int8 digit planes (quantized once per call); "
-                     "u8 x s8 -> s32 MMA (exact); fp32 output"}
+            "batch": 1, "tblk": cfg.tblk,
+            "step": ("lq_lift_gemv on this rank's rows + all-gather of the outputs" if shard
+                     else "lq_lift_gemv (lift + gemv)"),
+            "parallelism": f"rows{world}" if shard else f"replicas{world}",
+            "arith": "lift fp32; u as 32-bit fixed point in four int8 digit planes (quantized inside each "
+                     "GEMV CTA); u8 x s8 -> s32 mma.sync (exact); fp32 output"}
 
 
 # ------------------------------------------------------------------ helpers
@@ -70,19 +73,28 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def source_digest(paths):
+    """sha256 prefix over the named source files, in order (comma-separated list)."""
+    import hashlib
+    h = hashlib.sha256()
+    for p in paths.split(","):
+        with open(os.path.join(ROOT, p), "rb") as src:
+            h.update(src.read())
+    return h.hexdigest()[:16]
+
+
 def profiled_traffic(kernel_key):
     """DRAM bytes per launch from an ncu capture recorded in profiles/traffic.txt, or None
-    when absent or when the kernel source has changed since the capture (sha256 prefix)."""
-    import hashlib
+    when absent or when any source the kernel is built from has changed since the
+    capture (sha256 prefix over the listed files)."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         with open(path) as f:
             for line in f:
                 parts = line.split()
                 if len(parts) == 4 and parts[0] == kernel_key:
-                    with open(os.path.join(ROOT, parts[1]), "rb") as src:
-                        if hashlib.sha256(src.read()).hexdigest()[:16] != parts[2]:
-                            return None
+                    if source_digest(parts[1]) != parts[2]:
+                        return None
                     return float(parts[3])
     except OSError:
         pass
@@ -235,6 +247,37 @@ class DecodeLayer:
         return self.cfg.out * self.cfg.K // 8
 
 
+def shard_rows(out, world, rank):
+    from bit_lifted_gemm_b200.sharded import row_range
+    r0, r1 = row_range(out, world, rank)
+    return r1 - r0
+
+
+class ShardedLayer:
+    """Row-sharded decode (bit_lifted_gemm_b200.sharded.ShardedDecode), one
+    instance per weight copy: every rank lifts the whole batch, contracts its
+    rows and all-gathers the outputs."""
+
+    def __init__(self, lq, cfg, copies, torch, world, rank):
+        from bit_lifted_gemm_b200.sharded import ShardedDecode
+        L = make_layer(cfg, 1)
+        dev = torch.device("cuda")
+        pk = torch.from_numpy(L.packed.view(np.int32))
+        s = torch.from_numpy(L.s)
+        tinv = torch.from_numpy(L.tinv).to(dev) if L.tinv is not None else None
+        M = torch.from_numpy(L.M).to(dev)
+        self.parts = [ShardedDecode(pk, s, M, cfg.K, tinv=tinv, batch=1) for _ in range(copies)]
+        a = torch.from_numpy(L.a.view(np.int16)).to(dev).view(torch.bfloat16) if L.a_dtype == "bf16" \
+            else torch.from_numpy(L.a).to(dev)
+        self.a = [a.clone() for _ in range(copies)]
+
+    def step(self, i):
+        self.parts[i].step(self.a[i])
+
+    def gemv_only(self, i):
+        self.parts[i].gemv_only()
+
+
 def copies_for(bytes_per_copy, l2_bytes):
     return max(STEPS_PER_GRAPH, int(np.ceil(3 * l2_bytes / bytes_per_copy)))
 
@@ -267,15 +310,6 @@ def time_graph(torch, graph, reps, per_rep):
     e1.record(st)
     e1.synchronize()
     return e0.elapsed_time(e1) / (reps * per_rep)
-
-
-def run_steps(torch, graph_full, graphs_single, steps):
-    """Replay exactly `steps` steps: full 16-step graphs, then single-step graphs."""
-    full, rem = divmod(steps, STEPS_PER_GRAPH)
-    for _ in range(full):
-        graph_full.replay()
-    for i in range(rem):
-        graphs_single[i].replay()
 
 
 # ------------------------------------------------------------------ oracle on host cores
@@ -476,18 +510,67 @@ def bench_prefill(torch, lq, name, tokens, reps=10):
             "layer_tokens_per_s": tokens / ((ms_lift + ms_gemm) * 1e-3)}
 
 
+GRAPH_STEPS = 1024      # steps per CUDA graph of the timed region
+GEMV_LAUNCHES = 2048    # GEMV-alone launches behind the roofline, whatever --steps is
+LAUNCHES_PER_STEP = 3   # lift, u quantizer, GEMV contraction
+
+
+def spawn_ranks(args):
+    """`--gpus N` with N > 1 outside a launcher: start N ranks with torch.distributed.run."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    os.execv(sys.executable, cmd)
+
+
+class StepPlan:
+    """Exactly n steps as replays of one GRAPH_STEPS-step graph and one graph of
+    the remainder; step i of the run uses weight copy i % copies."""
+
+    def __init__(self, torch, fn, n, copies, full=None):
+        self.n = n
+        self.full = full if full is not None else (
+            capture(torch, fn, GRAPH_STEPS) if n >= GRAPH_STEPS else None)
+        self.nfull, rem = divmod(n, GRAPH_STEPS)
+        # the remainder continues the rotation where the full graphs leave it
+        off = (self.nfull * GRAPH_STEPS) % copies
+        self.rem = capture(torch, lambda i: fn((off + i) % copies), rem) if rem else None
+
+    def replay(self):
+        for _ in range(self.nfull):
+            self.full.replay()
+        if self.rem is not None:
+            self.rem.replay()
+
+    def warm(self):
+        for g in (self.full, self.rem):
+            if g is not None:
+                g.replay()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=160000)
+    ap.add_argument("--steps", type=int, default=100000)
     ap.add_argument("--warmup", type=int, default=2000)
     ap.add_argument("--impl", default="lq", choices=["lq", "reference"])
     ap.add_argument("--workload", default="decode_lq24_10")
+    ap.add_argument("--shard", default="none", choices=["none", "rows"],
+                    help="rows: one layer split by output rows over the ranks (strong scaling)")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary sweeps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.steps < 1:
+        raise SystemExit("--steps must be at least 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        spawn_ranks(args)
     world, rank, local = dist_setup()
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch one rank per GPU")
 
     if args.impl == "reference":
         reference_arm(args, world, rank)
@@ -507,32 +590,25 @@ def main():
     l2 = getattr(props, "L2_cache_size", 126 * 2**20) or 126 * 2**20
     cfg = CONFIGS[args.workload]
     probe = make_layer(cfg, 1, packed=False)
-    per_copy = cfg.out * cfg.K // 8 + (probe.tinv.nbytes if probe.tinv is not None else 0) + 4 * cfg.out
+    shard = args.shard == "rows"
+    rows_here = shard_rows(cfg.out, world, rank) if shard else cfg.out
+    per_copy = rows_here * cfg.K // 8 + (probe.tinv.nbytes if probe.tinv is not None else 0) + 4 * rows_here
     copies = copies_for(per_copy, l2)
     copies = (copies + STEPS_PER_GRAPH - 1) // STEPS_PER_GRAPH * STEPS_PER_GRAPH
-    layer = DecodeLayer(lq, cfg, 1, copies, torch)
+    layer = (ShardedLayer(lq, cfg, copies, torch, world, rank) if shard
+             else DecodeLayer(lq, cfg, 1, copies, torch))
+    step = layer.step
 
-    # one graph per 16-step block of distinct weight copies
-    blocks = copies // STEPS_PER_GRAPH
-    g_full = [capture(torch, lambda i, b=b: layer.step(b * STEPS_PER_GRAPH + i), STEPS_PER_GRAPH)
-              for b in range(blocks)]
-    g_single = [capture(torch, lambda i, j=j: layer.step(j), 1) for j in range(STEPS_PER_GRAPH)]
-    g_gemv = [capture(torch, lambda i, b=b: layer.gemv_only(b * STEPS_PER_GRAPH + i), STEPS_PER_GRAPH)
-              for b in range(blocks)]
-    g_e2e = [capture(torch, lambda i, b=b: layer.step(b * STEPS_PER_GRAPH + i, with_copies=True), STEPS_PER_GRAPH)
-             for b in range(blocks)]
-    g_zc = [capture(torch, lambda i, b=b: layer.step_zero_copy(b * STEPS_PER_GRAPH + i), STEPS_PER_GRAPH)
-            for b in range(blocks)]
-
-    def replay_steps(graphs, n):
-        full, rem = divmod(n, STEPS_PER_GRAPH)
-        for k in range(full):
-            graphs[k % len(graphs)].replay()
-        for i in range(rem):
-            g_single[i].replay()
+    plan = StepPlan(torch, lambda i: step(i % copies), args.steps, copies)
+    warm = StepPlan(torch, lambda i: step(i % copies), args.warmup, copies, full=plan.full)
+    g_gemv = capture(torch, lambda i: layer.gemv_only(i % copies), GEMV_LAUNCHES // 16)
+    e_plan = None if shard else StepPlan(torch, lambda i: layer.step_zero_copy(i % copies), args.steps, copies)
+    c_plan = None if shard else StepPlan(torch, lambda i: layer.step(i % copies, with_copies=True),
+                                         args.steps, copies)
 
     st = torch.cuda.current_stream()
-    replay_steps(g_full, args.warmup)
+    warm.replay()
+    plan.warm()
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
@@ -542,7 +618,7 @@ def main():
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler.mark("begin")
     e0.record(st)
-    replay_steps(g_full, args.steps)
+    plan.replay()
     e1.record(st)
     e1.synchronize()
     sampler.mark("end")
@@ -551,76 +627,87 @@ def main():
     ms_total = max_over_ranks(e0.elapsed_time(e1), world, device)
     clocks = sampler.stop()
     ms_per_step = ms_total / args.steps
-    launches = 2 * args.steps
+    launches = LAUNCHES_PER_STEP * args.steps
 
-    # dominant kernel alone (same stream, right after the step region)
-    reps = max(1, min(2000, args.steps // STEPS_PER_GRAPH))
+    # dominant kernel alone (same stream, after the step region): a fixed number of launches
+    g_gemv.replay()
+    torch.cuda.synchronize()
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2.record(st)
-    for k in range(reps):
-        g_gemv[k % blocks].replay()
+    for _ in range(16):
+        g_gemv.replay()
     e3.record(st)
     e3.synchronize()
-    gemv_us = e2.elapsed_time(e3) * 1e3 / (reps * STEPS_PER_GRAPH)
-    gemv_us = max_over_ranks(gemv_us, world, device)
+    gemv_us = max_over_ranks(e2.elapsed_time(e3) * 1e3 / GEMV_LAUNCHES, world, device)
 
-    # end to end: pinned host activations in, output back to the host, every step
-    e_steps = max(STEPS_PER_GRAPH, min(args.steps, 16000) // STEPS_PER_GRAPH * STEPS_PER_GRAPH)
-    barrier(world, device)
-    torch.cuda.synchronize()
-    def time_e2e(graphs):
+    def time_plan(p):
+        p.warm()
         barrier(world, device)
         torch.cuda.synchronize()
         e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e4.record(st)
-        for k in range(e_steps // STEPS_PER_GRAPH):
-            graphs[k % blocks].replay()
+        p.replay()
         e5.record(st)
         e5.synchronize()
-        return max_over_ranks(e4.elapsed_time(e5), world, device) / e_steps
+        return max_over_ranks(e4.elapsed_time(e5), world, device) / p.n
 
-    ms_e2e_copies = time_e2e(g_e2e)
-    ms_e2e = time_e2e(g_zc)
-    torch.cuda.synchronize()
-    for i in (0, copies - 1):   # zero-copy output equals the device step's, bit for bit
-        if not torch.equal(layer.o_host[i], layer.o[i].cpu()):
-            raise RuntimeError(f"zero-copy step {i} differs from the device step")
-
-    packed_bytes = layer.packed_bytes
-    value = world * packed_bytes / (ms_per_step * 1e-3) / 1e9
-    achieved = packed_bytes / (gemv_us * 1e-6) / 1e9
+    packed_bytes = cfg.out * cfg.K // 8          # the whole layer's signs, every step
+    local_bytes = rows_here * cfg.K // 8         # this rank's share
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    traffic = profiled_traffic("gemv_decode_lq24_10")
+    achieved = local_bytes / (gemv_us * 1e-6) / 1e9
+    if shard:
+        value = packed_bytes / (ms_per_step * 1e-3) / 1e9
+        e2e = {"value": None, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
+               "note": "row-sharded mode times the device path only"}
+    else:
+        ms_e2e = time_plan(e_plan)
+        ms_e2e_copies = time_plan(c_plan)
+        torch.cuda.synchronize()
+        for i in (0, copies - 1):   # zero-copy output equals the device step's, bit for bit
+            layer.step(i)
+            layer.step_zero_copy(i)
+            torch.cuda.synchronize()
+            if not torch.equal(layer.o_host[i], layer.o[i].cpu()):
+                raise RuntimeError(f"zero-copy step {i} differs from the device step")
+        value = world * packed_bytes / (ms_per_step * 1e-3) / 1e9
+        e2e = {"value": world * packed_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": int(layer.a[0].numel() * layer.a[0].element_size()),
+               "d2h_bytes_per_step": int(layer.o[0].numel() * 4), "ms_per_step": ms_e2e,
+               "mode": "zero-copy",
+               "note": "CUDA-graph replay of lq_lift_gemv on pinned host buffers: the lift loads the "
+                       "activations and the GEMV stores the output across the host link",
+               "copy_engine": {"value": world * packed_bytes / (ms_e2e_copies * 1e-3) / 1e9,
+                               "ms_per_step": ms_e2e_copies,
+                               "note": "H2D copy of the activations, lq_lift_gemv on device buffers, "
+                                       "D2H copy of the output"}}
+    traffic = profiled_traffic("gemv_decode_lq24_10") if (args.workload == "decode_lq24_10" and not shard) else None
+    config = dict(workload_config(cfg, args.workload, world, shard),
+                  l2=f"inputs larger than L2: {copies} rotating weight copies "
+                     f"({copies * per_copy / 1e6:.0f} MB vs L2 {l2 / 1e6:.0f} MB)",
+                  graphs=f"{plan.nfull} x {GRAPH_STEPS}-step graph + {plan.n % GRAPH_STEPS}-step graph")
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
-        "data": "synthetic",
-        "config": dict(workload_config(cfg, args.workload, world),
-                       l2=f"inputs larger than L2: {copies} rotating weight copies "
-                          f"({copies * per_copy / 1e6:.0f} MB vs L2 {l2 / 1e6:.0f} MB)"),
+        "higher_is_better": True, "scaling": "strong" if shard else "weak", "vs_baseline": None, "dtype": "i8",
+        "data": "synthetic", "config": config,
         "roofline": {"bound": "hbm", "kernel": "lq_gemv", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic, "peak_source": peaks_src,
-                     "avg_launch_us": gemv_us, "algorithmic_bytes_per_launch": packed_bytes},
-        "e2e": {"value": world * packed_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
-                "h2d_bytes_per_step": int(layer.a[0].numel() * layer.a[0].element_size()),
-                "d2h_bytes_per_step": int(layer.o[0].numel() * 4), "ms_per_step": ms_e2e,
-                "mode": "zero-copy",
-                "note": "CUDA-graph replay of lq_lift_gemv on pinned host buffers: the lift loads the "
-                        "activations and the GEMV stores the output across the host link",
-                "copy_engine": {"value": world * packed_bytes / (ms_e2e_copies * 1e-3) / 1e9,
-                                "ms_per_step": ms_e2e_copies,
-                                "note": "H2D copy of the activations, lq_lift_gemv on device buffers, "
-                                        "D2H copy of the output"}},
+                     "avg_launch_us": gemv_us, "launches_timed": GEMV_LAUNCHES,
+                     "algorithmic_bytes_per_launch": local_bytes},
+        "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
     }
+    if shard:
+        result["multi_gpu"] = ("unmeasured on hardware beyond one GPU" if world == 1 else
+                               f"{world} ranks, all-gather of the outputs over NCCL")
 
     if rank == 0 and world == 1 and not args.no_extra:
         extra = {}
-        extra["prefill_lq24_10"] = bench_prefill(torch, lq, "prefill_lq24_10", 2048)
-        extra["prefill_lq24_10"]["frac_of_bf16_peak"] = (
-            extra["prefill_lq24_10"]["gemm_TFLOPs"] / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])))
+        pre = bench_prefill(torch, lq, "prefill_lq24_10", 2048)
+        bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        pre["frac_of_bf16_peak"] = pre["gemm_TFLOPs"] / bf16
+        extra["prefill_lq24_10"] = pre
         extra["decode_lq20_8"] = bench_decode_sweep(torch, lq, "decode_lq20_8", (1, 2, 4, 8, 16), l2)
         for D in (16, 19, 20, 22, 24):
             n = f"sweep_lq{D}_8"
@@ -628,7 +715,12 @@ def main():
                         "b64": bench_prefill(torch, lq, n, 64)}
         extra["kron_lq24_10"] = bench_kron(torch, lq, l2)
         extra["encode"] = bench_encode(torch, lq)
-        result["extra"] = extra
+        # the bulky record on a line of its own, before the headline
+        print(json.dumps({"extra": extra}), flush=True)
+        sweep = extra["decode_lq20_8"]
+        result["prefill"] = {"tflops": pre["gemm_TFLOPs"], "frac": pre["frac_of_bf16_peak"], "tokens": 2048,
+                             "peak_tflops": bf16}
+        result["decode_lq20_8_gemv_us"] = {b: round(v["gemv_us"], 2) for b, v in sweep.items()}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -642,7 +734,8 @@ def main():
         print(json.dumps(result), flush=True)
     if world > 1:
         import torch.distributed as dist
-        del g_full, g_single, g_gemv, g_e2e, g_zc
+        del plan, warm, g_gemv, layer
+        torch.cuda.synchronize()
         dist.destroy_process_group()
 
 

@@ -1,25 +1,20 @@
-// Decode-path plan and workspace layout, shared by the u quantizer
-// (lq_quant.cu), the two decode contraction kernels (lq_gemv.cu on mma.sync,
-// lq_gemv_tc.cu on tcgen05) and the C ABI (lq_api.cu).
+// Decode-path plan and workspace layout, shared by the quantizer of the
+// tensor-core path (lq_quant.cu), the two decode contraction kernels
+// (lq_gemv.cu on mma.sync, lq_gemv_tc.cu on tcgen05) and the C ABI (lq_api.cu).
 //
-// The decode contraction runs on integer tensor cores. Each column c of the
-// lifted activations u is quantized once per call, by the quantizer, to 32-bit
-// fixed point with one power-of-two scale:
-//
-//   u_q[c][k] = round(u[c][k] * 2^F_c),   |u_q| <= 2^30,
-//
-// held as four balanced int8 digit planes u_q = d0 + 2^8 d1 + 2^16 d2 + 2^24 d3
-// (the bytes of (u_q + 0x80808080) ^ 0x80808080). An element's rounding error is
-// at most 2^-31 of the column's largest |u|. The contraction kernels add the
+// mma.sync path (up to three columns): each CTA quantizes the K range of its
+// launch itself, column by column, to 32-bit fixed point with one
+// power-of-two scale, u_q[c][k] = round(u[c][k] * 2^F_c), |u_q| <= 2^30, held
+// as four balanced int8 digit planes u_q = d0 + 2^8 d1 + 2^16 d2 + 2^24 d3 (the
+// bytes of (u_q + 0x80808080) ^ 0x80808080). An element's rounding error is at
+// most 2^-31 of the largest |u| of its column and K range. The kernel adds the
 // digits of the set bits exactly in integers (sum sigma u_q = 2 sum_{bit=1} u_q
-// - sum u_q), so the only rounding is this quantization and the final fp32 store.
+// - sum u_q), so the only rounding is this quantization and the final stores.
+// Columns holding a NaN are written as NaN; columns holding +-Inf are
+// contracted on their Inf pattern (lq_gemv.cu).
 //
-// Columns holding a NaN are written as NaN. Columns holding +-Inf (and no NaN)
-// are contracted on their Inf pattern instead: u_q = +1 at +Inf, -1 at -Inf,
-// 0 elsewhere, F = 0. For a row r, S = sum sigma u_q counts the +Inf terms minus
-// the -Inf terms of sigma[r][k] * u[k], n the Inf elements, so the IEEE sum of
-// the row is +Inf (S == n), -Inf (S == -n) or NaN (anything else) -- the same as
-// an exact sum in floating point.
+// tcgen05 path (four or more columns): the block-scaled 4-bit form below,
+// quantized once per call into the workspace.
 #pragma once
 
 #include <stddef.h>
@@ -28,23 +23,10 @@
 namespace lq {
 
 constexpr int kPlanes = 4;       // int8 digit planes of the 32-bit fixed point
-constexpr int kStepWords = 16;   // words of K (512 elements) per step sum
+constexpr int kStepWords = 16;   // words of K per weight step of the mma.sync kernel
 constexpr int kMaxColsPass = 2;  // batch columns per mma.sync pass (8 digit columns = one n8 tile)
 
 enum : int { kColFinite = 0, kColInf = 1, kColNaN = 2 };
-
-struct ColHeader {
-    int F;     // u_q = round(u * 2^F) (finite columns)
-    int mode;  // kColFinite, kColInf or kColNaN
-    int pad0, pad1;
-};
-
-// Per (column, 16-word step of K): sum of u_q and the number of +-Inf elements.
-struct StepSum {
-    long long S;
-    int ninf;
-    int pad;
-};
 
 // 16-byte chunk index of word pair (x, x+1), x even, in an mma.sync digit
 // plane: the four chunks from 2x + x/4 (the x/4 skew keeps a quarter-warp's
@@ -86,14 +68,14 @@ constexpr uint32_t kInfoExp = 0x1ffu, kInfoNaN = 1u << 9, kInfoInf = 1u << 10;
 
 // Launch plan of one decode contraction and the layout of its workspace.
 struct DecodePlan {
-    int out, K, kw, batch, nsteps;
+    int out, K, kw, batch;
     bool tc;  // block-scaled tcgen05 kernel (else mma.sync on 32-bit fixed point)
 
     // ---- mma.sync kernel (lq_gemv.cu)
     int grid, ts, stages, cols, npass, kwc, nchunk, pitch, maxgroups;
-    bool tma;
+    bool tma, ustage;  // weights through TMA rings; u staged by TMA (else read directly)
     size_t smem;
-    size_t image_bytes;  // digit planes of one (pass, K chunk): kPlanes * cols * pitch * 16
+    size_t image_bytes;  // shared-memory digit planes of one (pass, K chunk): kPlanes * cols * pitch * 16
 
     // ---- tcgen05 kernel (lq_gemv_tc.cu)
     int tc_grid, tc_bpad, tc_n, tc_groups, tc_stages, tc_maxcontrib, tc_nq, tc_nacc, tc_nss, tc_nsa, tc_mt;
@@ -103,25 +85,12 @@ struct DecodePlan {
     size_t row_bytes;       // bytes of one B row (one plane of one column): K / 2
 
     // ---- workspace (byte offsets from its 256-byte aligned base)
-    //   mma.sync: hdr = ColHeader[batch], steps = StepSum[batch][nsteps], planes = images
+    //   mma.sync: none used (256 bytes are still asked for)
     //   tcgen05:  hdr = column summaries uint32 [batch][tc_nqp], steps = word deltas
     //             uint8 [batch][tc_kwp], planes = B rows [kMxPlanes * tc_bpad][K / 2] (row p * tc_bpad + c),
     //             count = group counters, slots = split partial sums
     size_t off_hdr, off_steps, off_planes, off_count, off_slots, bytes;
 };
-
-// The digit register (j, x): bytes i = 0..3 hold the digits of elements
-// j + 8 i of word x (the same K order as the sign-bit masks of a word).
-// Byte offset of register (j, x) of plane `pl` of column c in the mma.sync
-// images: image (pass c / cols, chunk x / kwc), plane 4 (c % cols) + pl, chunk
-// run of pair (x & ~1), word 2 (j & 1) + (x & 1) of chunk j / 2.
-__host__ __device__ inline size_t mma_digit_offset(const DecodePlan& p, int c, int pl, int x, int j) {
-    const int pass = c / p.cols, cl = c % p.cols;
-    const int q = x / p.kwc, xl = x - q * p.kwc;
-    const size_t image = (size_t)(pass * p.nchunk + q) * p.image_bytes;
-    const size_t plane = (size_t)(kPlanes * cl + pl) * p.pitch * 16;
-    return image + plane + (size_t)(chunkpos(xl & ~1) + (j >> 1)) * 16 + (size_t)(2 * (j & 1) + (xl & 1)) * 4;
-}
 
 // Host: the plan for (out, K, batch); .bytes == 0 if no plan fits.
 DecodePlan make_decode_plan(int out, int K, int batch);

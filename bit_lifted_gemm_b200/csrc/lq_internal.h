@@ -65,7 +65,6 @@ struct DecodePlan;
 // The quantizers (lq_quant.cu): 32-bit fixed point for the mma.sync kernel
 // (it also clears `nzero` words at `zero`), block-scaled e2m1 digits for the
 // tcgen05 kernel (it also clears the kernel's group counters).
-cudaError_t launch_quant(const float* u, const DecodePlan& p, void* ws, unsigned* zero, int nzero, cudaStream_t st);
 cudaError_t launch_quant_mx(const float* u, const DecodePlan& p, void* ws, cudaStream_t st);
 // The tcgen05 contraction (lq_gemv_tc.cu): plan_tc fills the tc_* fields and
 // returns whether the shape takes that kernel; tc_slot_bytes is the size of its

@@ -41,11 +41,15 @@ class ShardedDecode:
 
     packed [out][K/32] (int32 storage of uint32) and s [out] may live on the host or
     the device; this rank copies its rows to the current device. M [d][D] and the
-    whitening inverse tinv (or None) are replicated."""
+    whitening inverse tinv (or None) are replicated. The GEMV workspace is
+    allocated once. Given `batch`, the lifted activations, the local output, the
+    gather buffer and the assembled output are allocated here too, and step()
+    launches no allocation (it can be captured in a CUDA graph)."""
 
-    def __init__(self, packed, s, M, K, tinv=None, group=None):
+    def __init__(self, packed, s, M, K, tinv=None, group=None, batch=None):
         import torch
         import torch.distributed as dist
+        from . import gemv_workspace
         self.group = group
         self.dist = dist.is_initialized()
         self.world = dist.get_world_size(group) if self.dist else 1
@@ -54,20 +58,58 @@ class ShardedDecode:
         r0, r1 = row_range(out, self.world, self.rank)
         h = shard_height(out, self.world)
         dev = torch.device("cuda", torch.cuda.current_device())
-        self.out, self.K, self.h = out, K, h
+        self.out, self.K, self.h, self.dev = out, K, h, dev
         self.packed = torch.zeros((h, K // 32), dtype=torch.int32, device=dev)
         self.packed[: r1 - r0].copy_(packed[r0:r1])
         self.s = torch.zeros(h, dtype=torch.float32, device=dev)
         self.s[: r1 - r0].copy_(s[r0:r1])
         self.M = M.to(dev).contiguous()
         self.tinv = None if tinv is None else tinv.to(dev).contiguous()
+        self._ws = {}
+        self.batch = batch
+        if batch is not None:
+            self.u = torch.empty((batch, K), dtype=torch.float32, device=dev)
+            self.o_local = torch.empty((batch, h), dtype=torch.float32, device=dev)
+            self.gathered = (torch.empty((self.world, batch, h), dtype=torch.float32, device=dev)
+                             if self.dist else None)
+            self._workspace(batch)
+
+    def _workspace(self, batch):
+        from . import gemv_workspace
+        if batch not in self._ws:
+            self._ws[batch] = gemv_workspace(self.h, self.K, batch, self.dev)
+        return self._ws[batch]
+
+    def step(self, a):
+        """a [batch][in] on this rank's device (batch as given at construction):
+        lift, GEMV on this rank's rows, all-gather of the shard outputs into
+        self.gathered [world][batch][h] (with no process group the local output
+        is the whole of o); assembled() gives o."""
+        import torch.distributed as dist
+        from . import lift_gemv
+        lift_gemv(a, self.M, self.packed, self.s, self.K, tinv=self.tinv, u=self.u, out=self.o_local,
+                  workspace=self._ws[self.batch])
+        if self.dist:
+            dist.all_gather_into_tensor(self.gathered, self.o_local, group=self.group)
+
+    def gemv_only(self):
+        """The GEMV on this rank's rows from the lifted activations of the last step."""
+        from . import gemv
+        gemv(self.packed, self.s, self.u, out=self.o_local, workspace=self._ws[self.batch])
+
+    def assembled(self):
+        """o [batch][out] from the last step's gathered shard outputs."""
+        if not self.dist:
+            return self.o_local[:, : self.out]
+        return assemble(list(self.gathered.unbind(0)), self.out, self.world)
 
     def __call__(self, a):
         """a [batch][in] on this rank's device -> o [batch][out] (every rank gets all of o)."""
         import torch
         import torch.distributed as dist
         from . import lift_gemv
-        _, o_local = lift_gemv(a, self.M, self.packed, self.s, self.K, tinv=self.tinv)
+        _, o_local = lift_gemv(a, self.M, self.packed, self.s, self.K, tinv=self.tinv,
+                               workspace=self._workspace(int(a.shape[0])))
         if not self.dist:
             return o_local[:, : self.out]
         pieces = [torch.empty_like(o_local) for _ in range(self.world)]

@@ -593,6 +593,9 @@ def test_sharded_decode_single_gpu(lq):
     _, want = lq.lift_gemv(a, dev(L.M), dev(L.packed), dev(L.s), K, tinv=dev(L.tinv))
     sd = ShardedDecode(packed_h, s_h, dev(L.M), K, tinv=dev(L.tinv))
     assert np.array_equal(host(sd(a)), host(want))
+    sdb = ShardedDecode(packed_h, s_h, dev(L.M), K, tinv=dev(L.tinv), batch=4)  # preallocated step
+    sdb.step(a)
+    assert np.array_equal(host(sdb.assembled()), host(want))
     sock = socket.socket()
     sock.bind(("127.0.0.1", 0))
     port = sock.getsockname()[1]
@@ -604,6 +607,10 @@ def test_sharded_decode_single_gpu(lq):
         got = sd1(a)
         torch.cuda.synchronize()
         assert np.array_equal(host(got), host(want))
+        sd2 = ShardedDecode(packed_h, s_h, dev(L.M), K, tinv=dev(L.tinv), batch=4)
+        sd2.step(a)  # all_gather_into_tensor into the preallocated buffer
+        torch.cuda.synchronize()
+        assert np.array_equal(host(sd2.assembled()), host(want))
     finally:
         dist.destroy_process_group()
 
