@@ -405,21 +405,39 @@ __global__ void __maxnreg__(128)  // 384 threads: leaves registers for a lift be
             const int mode = c == 0 ? cmode[0] : cmode[kMaxColsPass - 1];
             const float sa = c == 0 ? csa[0] : csa[kMaxColsPass - 1], sb = c == 0 ? csb[0] : csb[kMaxColsPass - 1];
             uint8_t* pc = planes8 + (size_t)(kPlanes * c) * p.pitch * 16;
+            const size_t pstride = (size_t)p.pitch * 16;
             long long qs = 0;
             int ni = 0;
+            if (mode == kColFinite) {  // the common case, without per-element mode tests
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int q0 = quant_elem(v[rd][j], mode, sa, sb), q1 = quant_elem(v[rd][j + 8], mode, sa, sb);
-                const int q2 = quant_elem(v[rd][j + 16], mode, sa, sb), q3 = quant_elem(v[rd][j + 24], mode, sa, sb);
-                uint32_t P[kPlanes];
-                digit_regs(q0, q1, q2, q3, P);
-                const int off = digit_offset(j, xl);
+                for (int j = 0; j < 8; ++j) {
+                    const int q0 = __float2int_rn((v[rd][j] * sa) * sb);
+                    const int q1 = __float2int_rn((v[rd][j + 8] * sa) * sb);
+                    const int q2 = __float2int_rn((v[rd][j + 16] * sa) * sb);
+                    const int q3 = __float2int_rn((v[rd][j + 24] * sa) * sb);
+                    uint32_t P[kPlanes];
+                    digit_regs(q0, q1, q2, q3, P);
+                    const int off = digit_offset(j, xl);
 #pragma unroll
-                for (int pl = 0; pl < kPlanes; ++pl)
-                    *reinterpret_cast<uint32_t*>(pc + (size_t)pl * p.pitch * 16 + off) = P[pl];
-                qs += (long long)q0 + q1 + q2 + q3;
-                ni += (int)isinf(v[rd][j]) + (int)isinf(v[rd][j + 8]) + (int)isinf(v[rd][j + 16]) +
-                      (int)isinf(v[rd][j + 24]);
+                    for (int pl = 0; pl < kPlanes; ++pl) *reinterpret_cast<uint32_t*>(pc + pl * pstride + off) = P[pl];
+                    // |q0 + q1| <= 2^31 fits unsigned 32-bit arithmetic exactly as a signed 33-bit value
+                    qs += (long long)(q0 + (long long)q1) + (long long)(q2 + (long long)q3);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int q0 = quant_elem(v[rd][j], mode, sa, sb), q1 = quant_elem(v[rd][j + 8], mode, sa, sb);
+                    const int q2 = quant_elem(v[rd][j + 16], mode, sa, sb);
+                    const int q3 = quant_elem(v[rd][j + 24], mode, sa, sb);
+                    uint32_t P[kPlanes];
+                    digit_regs(q0, q1, q2, q3, P);
+                    const int off = digit_offset(j, xl);
+#pragma unroll
+                    for (int pl = 0; pl < kPlanes; ++pl) *reinterpret_cast<uint32_t*>(pc + pl * pstride + off) = P[pl];
+                    qs += (long long)q0 + q1 + q2 + q3;
+                    ni += (int)isinf(v[rd][j]) + (int)isinf(v[rd][j + 8]) + (int)isinf(v[rd][j + 16]) +
+                          (int)isinf(v[rd][j + 24]);
+                }
             }
             add_sum(c, qs, ni);
         }
