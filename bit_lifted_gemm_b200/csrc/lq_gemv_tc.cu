@@ -194,22 +194,24 @@ __device__ __forceinline__ uint32_t idesc_mxf4(int N) {
     return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | (8u << 24);
 }
 
-// Walks a CTA's sub-stages: unit -> (group, sub-stage), the index of its
+// Walks a CTA's sub-stages: unit -> (group, sub-stage), the index ks of its
 // shared-memory stage in the CTA's sequence (a new stage starts at every
-// 32-word boundary and at every group), and whether it is the last sub-stage
-// of that stage or of its group segment.
+// 32-word boundary and at every group) with its ring slot ks % nss and phase
+// (ks / nss) & 1 kept incrementally, and whether it is the last sub-stage of
+// that stage or of its group segment.
 struct Walker {
     long long u0, u1;
-    int nsub;
+    int nsub, nss;
     long long g;
-    int sub, ks;
-    __device__ void init(long long a, long long b, int n) {
+    int sub, ks, slot, phase;
+    __device__ void init(long long a, long long b, int n, int stages) {
         u0 = a;
         u1 = b;
         nsub = n;
+        nss = stages;
         g = a / n;
         sub = (int)(a - g * n);
-        ks = 0;
+        ks = slot = phase = 0;
     }
     __device__ bool seg_first(long long u) const { return u == u0 || sub == 0; }
     __device__ bool seg_last(long long u) const { return u + 1 == u1 || sub + 1 == nsub; }
@@ -222,7 +224,28 @@ struct Walker {
         } else {
             ++sub;
         }
-        ks += new_stage ? 1 : 0;
+        if (new_stage) {
+            ++ks;
+            if (++slot == nss) {
+                slot = 0;
+                phase ^= 1;
+            }
+        }
+    }
+};
+
+// Index and phase of a ring of n slots, advanced one use at a time.
+struct Ring {
+    int idx, phase, n;
+    __device__ void init(int slots) {
+        idx = phase = 0;
+        n = slots;
+    }
+    __device__ void next() {
+        if (++idx == n) {
+            idx = 0;
+            phase ^= 1;
+        }
     }
 };
 
@@ -292,16 +315,14 @@ __global__ void __launch_bounds__(tc_threads(MT), 1)
         // ================================================================ TMA producer
         if (lane == 0) {
             Walker wk;
-            wk.init(u0, u1, p.nsub);
-            auto issue_w = [&](int ks, long long g, int stg) {
-                const int slot = ks % nss;
+            wk.init(u0, u1, p.nsub, nss);
+            auto issue_w = [&](int slot, long long g, int stg) {
                 mbar_arrive_expect_tx(full_w + 8 * slot, MT * kWTile);
                 for (int t = 0; t < MT; ++t)
                     tma_load_2d(smem_addr(smem + L.w + ((size_t)slot * MT + t) * kWTile), &wmap, stg * kStageW,
                                 (int)(g * kRG) + 128 * t, full_w + 8 * slot);
             };
-            auto issue_b = [&](int ks, int stg) {
-                const int slot = ks % nss;
+            auto issue_b = [&](int slot, int stg) {
                 const uint32_t ib = smem_addr(smem + L.info + slot * L.istage);
                 mbar_arrive_expect_tx(full_b + 8 * slot, (uint32_t)(L.bstage + p.batch * (kStageW + 16)));
                 tma_load_3d(smem_addr(smem + L.b + slot * L.bstage), &bmap, 0, 0, stg * 4, full_b + 8 * slot);
@@ -325,15 +346,15 @@ __global__ void __launch_bounds__(tc_threads(MT), 1)
             int issued = 0;  // stages whose B was requested
             for (long long u = u0; u < u1; ++u) {
                 if (wk.stage_last(u)) {
-                    const int ks = wk.ks, slot = ks % nss;
+                    const int ks = wk.ks, slot = wk.slot;
                     if (ks >= nss) {
-                        if (!mbar_wait(freed + 8 * slot, ((ks / nss) - 1) & 1, p.status, kSpin)) {
+                        if (!mbar_wait(freed + 8 * slot, wk.phase ^ 1, p.status, kSpin)) {
                             *abort_flag = 1;
                             break;
                         }
-                        issue_w(ks, wk.g, wk.sub >> 2);
+                        issue_w(slot, wk.g, wk.sub >> 2);
                     }
-                    issue_b(ks, wk.sub >> 2);
+                    issue_b(slot, wk.sub >> 2);
                     issued = ks + 1;
                 }
                 wk.next(u);
@@ -380,13 +401,15 @@ __global__ void __launch_bounds__(tc_threads(MT), 1)
         }
         const int nrows4 = (p.N + 31) / 32;  // row blocks of 32 that hold B rows
         Walker wk;
-        wk.init(u0, u1, p.nsub);
+        wk.init(u0, u1, p.nsub, nss);
+        Ring ar;
+        ar.init(nsa);
         int i = 0;
-        for (long long u = u0; u < u1; ++u, ++i) {
-            const int ks = wk.ks, slot = ks % nss, j = wk.sub & 3, a = i % nsa;
-            bool ok = mbar_wait(full_w + 8 * slot, (ks / nss) & 1, p.status, kSpin);
-            ok = ok && mbar_wait(full_b + 8 * slot, (ks / nss) & 1, p.status, kSpin);
-            ok = ok && (i < nsa || mbar_wait(a_empty + 8 * a, ((i / nsa) - 1) & 1, p.status, kSpin));
+        for (long long u = u0; u < u1; ++u, ++i, ar.next()) {
+            const int slot = wk.slot, j = wk.sub & 3, a = ar.idx;
+            bool ok = mbar_wait(full_w + 8 * slot, wk.phase, p.status, kSpin);
+            ok = ok && mbar_wait(full_b + 8 * slot, wk.phase, p.status, kSpin);
+            ok = ok && (i < nsa || mbar_wait(a_empty + 8 * a, ar.phase ^ 1, p.status, kSpin));
             if (!__all_sync(0xffffffffu, ok) || *abort_flag) {  // tcgen05.st is warp-collective
                 *abort_flag = 1;
                 break;
@@ -418,15 +441,26 @@ __global__ void __launch_bounds__(tc_threads(MT), 1)
             const uint32_t* ssm = reinterpret_cast<const uint32_t*>(dsm + L.isumm);
             uint32_t sf[8] = {0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu,
                               0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu};
+            // every row block's loads first (rows without a B row read column 0)
+            uint32_t dlv[kRB], elv[kRB];
+#pragma unroll
+            for (int c4 = 0; c4 < kRB; ++c4) {
+                dlv[c4] = *reinterpret_cast<const uint32_t*>(dsm + rc[c4] * kStageW + 8 * j + 4 * k);
+                elv[c4] = ssm[4 * rc[c4] + j] & kInfoExp;
+            }
 #pragma unroll
             for (int c4 = 0; c4 < kRB; ++c4) {
                 uint32_t e4 = 0x7F7F7F7Fu;  // rows without a B row: any finite scale
                 if (c4 < nrows4 && rmode[c4] >= 0) {
-                    const uint32_t dl = *reinterpret_cast<const uint32_t*>(dsm + rc[c4] * kStageW + 8 * j + 4 * k);
+                    const uint32_t dl = dlv[c4];
                     if (rmode[c4] == kColFinite) {
                         // 2^(E - 1 - 3p - G_c): base 126 - 3p - (G_c - E_loc), less each word's delta
-                        const int base = max(0, rbase[c4] + (int)(ssm[4 * rc[c4] + j] & kInfoExp));
-                        e4 = __vsubus4((uint32_t)base * 0x01010101u, dl & 0x7F7F7F7Fu);
+                        const int base = max(0, rbase[c4] + (int)elv[c4]);
+                        // per byte max(0, base - delta), both below 128: (base | 0x80) - delta
+                        // stays within each byte, its bit 7 tells the sign
+                        const uint32_t t4 = ((uint32_t)base * 0x01010101u | 0x80808080u) - (dl & 0x7F7F7F7Fu);
+                        const uint32_t pos = (t4 >> 7) & 0x01010101u;
+                        e4 = t4 & 0x7F7F7F7Fu & (pos * 0xFFu);
                     } else if (rmode[c4] == kColInf) {
                         e4 = rp0[c4] ? ((dl >> 7) & 0x01010101u) * 127u : 0u;  // plane 0 of Inf words: 1.0
                     }
@@ -450,15 +484,16 @@ __global__ void __launch_bounds__(tc_threads(MT), 1)
             int buf = 0;
             int uses[2] = {0, 0};
             Walker wk;
-            wk.init(u0, u1, p.nsub);
-            int i = 0;
-            for (long long u = u0; u < u1; ++u, ++i) {
+            wk.init(u0, u1, p.nsub, nss);
+            Ring ar;
+            ar.init(nsa);
+            for (long long u = u0; u < u1; ++u, ar.next()) {
                 const bool first = wk.seg_first(u), last = wk.seg_last(u);
-                const int ks = wk.ks, slot = ks % nss, j = wk.sub & 3, a = i % nsa;
+                const int slot = wk.slot, j = wk.sub & 3, a = ar.idx;
                 bool ok = true;
                 if (first && uses[buf] > 0) ok = mbar_wait(acc_empty + 8 * buf, (uses[buf] - 1) & 1, p.status, kSpin);
-                ok = ok && mbar_wait(full_b + 8 * slot, (ks / nss) & 1, p.status, kSpin);
-                ok = ok && mbar_wait(a_full + 8 * a, (i / nsa) & 1, p.status, kSpin);
+                ok = ok && mbar_wait(full_b + 8 * slot, wk.phase, p.status, kSpin);
+                ok = ok && mbar_wait(a_full + 8 * a, ar.phase, p.status, kSpin);
                 if (!ok || *abort_flag) {
                     *abort_flag = 1;
                     break;
@@ -602,13 +637,19 @@ __global__ void __launch_bounds__(tc_threads(MT), 1)
                     const double* base = p.slots + ((size_t)(g * p.maxcontrib) * p.batch) * kRG;
 #pragma unroll 1
                     for (int t = 0; t < MT; ++t) {
+                        // slot order outside, columns inside: each round issues the
+                        // loads of every column at once
                         double sum[kCmax];
 #pragma unroll
-                        for (int c = 0; c < kCmax; ++c) {
-                            sum[c] = 0.0;
-                            if (c >= p.batch) continue;
-                            for (int jj = 0; jj < nc; ++jj)
-                                sum[c] += __ldcg(base + ((size_t)jj * p.batch + c) * kRG + t * 128 + 32 * q + lane);
+                        for (int c = 0; c < kCmax; ++c) sum[c] = 0.0;
+#pragma unroll 1
+                        for (int jj = 0; jj < nc; ++jj) {
+                            const double* sj = base + (size_t)jj * p.batch * kRG + t * 128 + 32 * q + lane;
+                            double x[kCmax];
+#pragma unroll
+                            for (int c = 0; c < kCmax; ++c) x[c] = c < p.batch ? __ldcg(sj + (size_t)c * kRG) : 0.0;
+#pragma unroll
+                            for (int c = 0; c < kCmax; ++c) sum[c] += x[c];
                         }
                         store_tile(t, sum);
                     }
