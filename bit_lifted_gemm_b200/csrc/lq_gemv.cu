@@ -4,13 +4,14 @@
 //
 //   o[c][r] = s[r] * sum_k sigma[r][k] u[c][k],   sigma = +1 if the bit is set.
 //
-// Up to three columns run on the mma.sync kernel of this file, which
+// One to three columns run on the mma.sync kernel of this file (three only
+// for layers under 40 MB of packed weights), which
 // quantizes u inside each CTA (a CTA contracts the whole K range of its launch,
 // so it needs every digit of it anyway; no extra launch, no scratch): each
 // column of the launch's K range becomes 32-bit fixed point with one
 // power-of-two scale, u_q = round(u * 2^F), |u_q| <= 2^30, held as four
 // balanced int8 digit planes (the bytes of (u_q + 0x80808080) ^ 0x80808080).
-// Four or more columns run on the tcgen05 kernel of lq_gemv_tc.cu, which reads
+// More columns run on the tcgen05 kernel of lq_gemv_tc.cu, which reads
 // every weight once for all columns, after the quantizer of lq_quant.cu has
 // written the block-scaled form of u once per call (lq_decode.h).
 //
@@ -849,12 +850,17 @@ DecodePlan make_decode_plan(int out, int K, int batch) {
     pl.kw = K / 32;
     pl.batch = batch;
     pl.row_bytes = (size_t)pl.kw * 16;
-    // Measured on B200 (13824 x 12288 and 28672 x 20480 layers): up to three
-    // columns the mma.sync kernel is faster, from four on the tensor-core
-    // kernel, which reads every weight once whatever the batch. Each takes the
-    // shapes the other cannot (the tensor-core kernel needs K a multiple of 256
-    // and at least 128 rows; the mma.sync kernel a word count its planes fit).
-    pl.tc = batch >= 4 && plan_tc(pl);
+    // Measured on B200 (13824 x 12288 and 28672 x 20480 layers, GEMV back to
+    // back): one and two columns are faster on the mma.sync kernel, four and
+    // more on the tensor-core kernel, which reads every weight once whatever
+    // the batch. At three columns mma.sync runs two passes (22.7 and 62.5 us)
+    // against a tensor-core launch of ~24 us plus ~0.28 us per MB of weights
+    // (30.0 and 44.8 us): the tensor-core kernel from 40 MB of packed weights.
+    // Each takes the shapes the other cannot (the tensor-core kernel needs K a
+    // multiple of 256 and at least 128 rows; the mma.sync kernel a word count
+    // its planes fit).
+    const double mbytes = (double)out * K / 8 / 1e6;
+    pl.tc = (batch >= 4 || (batch == 3 && mbytes >= 40.0)) && plan_tc(pl);
     if (!pl.tc && !plan_mma(pl) && !(pl.tc = plan_tc(pl))) return pl;
     size_t off = 0;
     if (pl.tc) {

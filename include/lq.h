@@ -165,13 +165,14 @@ LQ_API size_t lq_gemv_workspace_size(int out, int K, int batch);
  *   workspace : caller-owned device scratch of at least
  *               lq_gemv_workspace_size(out, K, batch) bytes, 256-byte aligned;
  *               its contents need no initialization and are overwritten.
- * Arithmetic: one to three columns run on mma.sync, which converts each
+ * Arithmetic: one or two columns (three below 40 MB of packed weights) run on
+ * mma.sync, which converts each
  * column of u (over the K range of each launch) to 32-bit fixed point with one
  * power-of-two scale -- an element's error is at most 2^-31 of the largest |u|
  * of its column and range -- and contracts the signs in exact integer
  * arithmetic; the result is within ~1e-7 relative (Frobenius) of the exact
- * value, and equal to it when u holds small integers. Four or more columns run
- * on tcgen05 block-scaled 4-bit MMAs, which read every weight once for all
+ * value, and equal to it when u holds small integers. More columns run on
+ * tcgen05 block-scaled 4-bit MMAs, which read every weight once for all
  * columns: u is converted once per call into the workspace, each 32-element
  * block with its own power-of-two scale to 21 bits (7 base-8 digits, error at
  * most 2^-21 of the block's largest |u|), accumulated in fp32 (~1e-6 relative).

@@ -248,7 +248,7 @@ def test_decode_lq24_10_full_size(lq):
     assert rel_err(o, want) <= 1e-5
 
 
-@pytest.mark.parametrize("batch", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("batch", [1, 2, 3, 4, 8, 16])  # three columns: the tensor-core path at this size
 def test_decode_lq20_8_sampled_rows(lq, batch):
     L = make_layer(CONFIGS["decode_lq20_8"], batch)
     u = _gpu_u(lq, L)
