@@ -201,6 +201,14 @@ int lq_lift_activations_kron(const void* a, int a_dtype, int batch, int in, cons
     if (sm < 0) return LQ_ERR_CUDA;
     if (sm == 0) return LQ_ERR_UNSUPPORTED;
     if (!all_device({a, r1, q1, q2, r2, M, u})) return LQ_ERR_INVALID_ARG;
+    if (lq::lift_kron_tc_supported(a_dtype == LQ_BF16, u_dtype == LQ_BF16, batch, in, n1, n2, d, D, K)) {
+        // prefill: both products on the tensor cores
+        int err = LQ_OK;
+        unsigned* status = status_word(&err);
+        if (!status) return err;
+        return from_cuda(lq::launch_lift_kron_tc(static_cast<const uint16_t*>(a), batch, in, r1, q1, n1, q2, n2, r2, M,
+                                                 d, D, u, K, status, static_cast<cudaStream_t>(stream)));
+    }
     return from_cuda(lq::launch_lift_kron(a, a_dtype == LQ_BF16, batch, in, r1, q1, n1, q2, n2, r2, M, d, D, u,
                                           u_dtype == LQ_BF16, K, static_cast<cudaStream_t>(stream)));
 }

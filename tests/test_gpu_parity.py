@@ -302,6 +302,11 @@ def _kron_oracle_u(a, a_dtype, M, kf, d, K, with_r=True):
     (48, 8, 4, 8, 3, "f32", "f32", True),         # d-blocks straddle rows of X; clusters of 4
     (640, 8, 10, 24, 70, "bf16", "bf16", True),   # 4 tokens per cluster, ragged last cluster, bf16 output
     (5120, 64, 10, 24, 40, "bf16", "bf16", True), # prefill-sized batch on the LQ-24/10 layer
+    # prefill on the tensor cores (bf16 in and out, 64 tokens or more)
+    (5120, 64, 10, 24, 300, "bf16", "bf16", True),  # 64 x 80 factors, ragged last 128-token tile
+    (8192, 64, 8, 20, 130, "bf16", "bf16", True),   # 64 x 128 factors, d = 8 blocks
+    (5120, 64, 10, 24, 200, "bf16", "bf16", False), # no diagonal factors
+    (4096, 64, 8, 16, 70, "bf16", "bf16", True),    # 64 x 64 factors, D = 2 d: K = 2 in exactly
 ])
 def test_lift_kron(lq, in_dim, n1, d, D, batch, a_dtype, u_dtype, with_r):
     """Lift with T^{-1} = diag(r2) (Q1 kron Q2) diag(r1) against the oracle."""
