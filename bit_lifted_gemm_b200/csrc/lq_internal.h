@@ -37,7 +37,7 @@ cudaError_t launch_lift_kron(const void* a, bool a_bf16, int batch, int in, cons
 
 // The same lift for prefill on tcgen05 (lq_lift_kron_tc.cu): bf16 activations
 // and u, at least 64 tokens, n1 <= 64, n2 a multiple of 16 up to 128, d <= 16
-// dividing n2, D >= 2 d even (u's rows hold the intermediate product first).
+// dividing n2, D >= 2 d a multiple of 4 (u's rows hold the intermediate product first).
 bool lift_kron_tc_supported(bool a_bf16, bool u_bf16, int batch, int in, int n1, int n2, int d, int D, int K);
 cudaError_t launch_lift_kron_tc(const uint16_t* a, int batch, int in, const float* r1, const float* q1, int n1,
                                 const float* q2, int n2, const float* r2, const float* M, int d, int D, void* u,

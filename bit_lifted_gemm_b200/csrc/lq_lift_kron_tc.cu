@@ -357,49 +357,42 @@ __global__ void __launch_bounds__(KZ_THREADS, 1)
 }
 
 // ============================================================================ a' = r2 o Q1 Z, lift
-// The lift of one token from its staged a' rows: thread (bi, ec) computes
-// outputs 2 ec and 2 ec + 1 of blocks bi, bi + nbi, ... (block b sits in row
-// b / bpr at column (b % bpr) d); M's two columns are in m0, m1. DD: d known
-// at compile time (0: generic). Consecutive threads write consecutive pairs of
-// a u row.
+// The lift of one token from its staged a' rows: thread (bi, e4) computes
+// outputs 4 e4 .. 4 e4 + 3 of blocks bi, bi + nbi, ... (block b sits in row
+// b / bpr at column (b % bpr) d); those four columns of M are in m. DD: d
+// known at compile time (0: generic). Consecutive threads write consecutive
+// 8-byte pieces of a u row.
 template <int DD>
-__device__ __forceinline__ void lift_token(const float* aps, int pitch, int bpr, int bi, int nbi, int nblocks, int ec,
-                                           int d, const float (&m0)[16], const float (&m1)[16], const float* r2,
-                                           __nv_bfloat16* urow, int D) {
+__device__ __forceinline__ void lift_token(const float* aps, int pitch, int bpr, int bi, int nbi, int nblocks, int e4,
+                                           int d, const float (&m)[4][16], const float* r2, __nv_bfloat16* urow,
+                                           int D) {
+    constexpr int DL = DD ? DD : 16;
+    const int dd = DD ? DD : d;
     int j1 = bi / bpr, off = bi - j1 * bpr;
     for (int b = bi; b < nblocks; b += nbi) {
-        const float* ar = aps + (size_t)j1 * pitch + off * (DD ? DD : d);
-        float s0 = 0.f, s1 = 0.f;
-        if constexpr (DD > 0) {
-            float av[DD];
-            if constexpr (DD % 2 == 0) {
+        const float* ar = aps + (size_t)j1 * pitch + off * dd;
+        float av[DL];
+        if constexpr (DD > 0 && DD % 2 == 0) {
 #pragma unroll
-                for (int i = 0; i < DD / 2; ++i) {
-                    const float2 f = *reinterpret_cast<const float2*>(ar + 2 * i);
-                    av[2 * i] = f.x;
-                    av[2 * i + 1] = f.y;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < DD; ++i) av[i] = ar[i];
-            }
-#pragma unroll
-            for (int i = 0; i < DD; ++i) {
-                s0 = fmaf(m0[i], av[i], s0);
-                s1 = fmaf(m1[i], av[i], s1);
+            for (int i = 0; i < DD / 2; ++i) {
+                const float2 f = *reinterpret_cast<const float2*>(ar + 2 * i);
+                av[2 * i] = f.x;
+                av[2 * i + 1] = f.y;
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                if (i < d) {
-                    const float av = ar[i];
-                    s0 = fmaf(m0[i], av, s0);
-                    s1 = fmaf(m1[i], av, s1);
-                }
-            }
+            for (int i = 0; i < DL; ++i) av[i] = i < dd ? ar[i] : 0.f;
         }
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < DL; ++i)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) s4[c] = fmaf(m[c][i], av[i], s4[c]);
         const float sc = r2 ? __ldg(r2 + b) : 1.f;
-        *reinterpret_cast<__nv_bfloat162*>(urow + (size_t)b * D + 2 * ec) = __floats2bfloat162_rn(s0 * sc, s1 * sc);
+        const __nv_bfloat162 h0 = __floats2bfloat162_rn(s4[0] * sc, s4[1] * sc);
+        const __nv_bfloat162 h1 = __floats2bfloat162_rn(s4[2] * sc, s4[3] * sc);
+        *reinterpret_cast<uint2*>(urow + (size_t)b * D + 4 * e4) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
         off += nbi;
         while (off >= bpr) {
             off -= bpr;
@@ -556,16 +549,15 @@ __global__ void __launch_bounds__(KY_THREADS, 1)
         mbar_arrive(aready);
         named_barrier_sync(1, 256);  // M is in shared memory for every worker
 
-        // the lift's thread map: pair ec of D / 2 output pairs and block offset bi;
-        // M's two columns of the pair stay in registers
-        const int nec = p.D / 2, nbi = 256 / nec;
+        // the lift's thread map: quad ec of D / 4 output quads and block offset bi;
+        // M's four columns of the quad stay in registers
+        const int nec = p.D / 4, nbi = 256 / nec;
         const int bi = w / nec, ec = w - bi * nec;
-        float m0[16], m1[16];
+        float m4[4][16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            m0[i] = (i < p.d && bi < nbi) ? Ms[i * p.D + 2 * ec] : 0.f;
-            m1[i] = (i < p.d && bi < nbi) ? Ms[i * p.D + 2 * ec + 1] : 0.f;
-        }
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) m4[c][i] = (i < p.d && bi < nbi) ? Ms[i * p.D + 4 * ec + c] : 0.f;
         const int bpr = p.n2 / p.d, nblocks = p.in / p.d;
         const int ngr = p.n2 / 8, nitem = p.n1p * ngr;
         const int q = warp & 3, half = (warp - 2) >> 2;  // warps 2..5: half 0, 6..9: half 1
@@ -641,13 +633,13 @@ __global__ void __launch_bounds__(KY_THREADS, 1)
             __nv_bfloat16* urow = p.u + (size_t)t * p.K;
             if (go && bi < nbi) {
                 if (p.d == 8)
-                    lift_token<8>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m0, m1, p.r2, urow, p.D);
+                    lift_token<8>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m4, p.r2, urow, p.D);
                 else if (p.d == 10)
-                    lift_token<10>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m0, m1, p.r2, urow, p.D);
+                    lift_token<10>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m4, p.r2, urow, p.D);
                 else if (p.d == 16)
-                    lift_token<16>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m0, m1, p.r2, urow, p.D);
+                    lift_token<16>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m4, p.r2, urow, p.D);
                 else
-                    lift_token<0>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m0, m1, p.r2, urow, p.D);
+                    lift_token<0>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m4, p.r2, urow, p.D);
             }
             // lifted columns past the last block are zero
             if (go)
@@ -712,7 +704,7 @@ int ky_depth(int n1p, int n2, int d, int D) {
 bool lift_kron_tc_supported(bool a_bf16, bool u_bf16, int batch, int in, int n1, int n2, int d, int D, int K) {
     if (!a_bf16 || !u_bf16 || batch < 64) return false;
     if (n1 < 8 || n1 > 64 || n2 < 16 || n2 > 128 || n2 % 16 != 0 || n1 * n2 != in) return false;
-    if (d < 1 || d > 16 || n2 % d != 0 || D < 2 * d || D % 2 != 0 || K < 2 * in) return false;
+    if (d < 1 || d > 16 || n2 % d != 0 || D < 2 * d || D % 4 != 0 || K < 2 * in) return false;
     const int n1p = round_up(n1, 16), n2p = n2;
     return kz_depth(n2p, (n2 + 63) / 64) > 0 && ky_depth(n1p, n2, d, D) > 0;
 }
