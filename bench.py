@@ -389,6 +389,10 @@ def bench_decode_sweep(torch, lq, name, batches, l2, reps=50):
         res[str(b)] = {"step_us": ms_step * 1e3, "gemv_us": ms_gemv * 1e3,
                        "gemv_GBps": layer.packed_bytes / (ms_gemv * 1e-3) / 1e9,
                        "layer_tokens_per_s": b / (ms_step * 1e-3)}
+        traffic = profiled_traffic(f"gemv_{name}_b{b}")
+        if traffic is not None:
+            # DRAM bytes of one GEMV launch (ncu) over the packed weights it streams
+            res[str(b)]["traffic_over_weights"] = traffic / (cfg.out * cfg.K // 8)
         del g, gg, layer
         torch.cuda.empty_cache()
     return res

@@ -46,14 +46,20 @@ struct Tile {
     static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * (A_STAGE + B_STAGE) + 256;
 };
 // The variant for short token runs keeps the A stages in TMEM after the
-// accumulator (the unpackers store them with tcgen05.st; no A traffic through
+// accumulators (the unpackers store them with tcgen05.st; no A traffic through
 // shared memory): measured faster for 64-token tiles, slower for 256-token ones.
-template <int BN>
+// Its k-steps alternate between NI issuing threads in separate warps, each with
+// an accumulator of its own: one thread's commits complete one after another,
+// ~400 clocks apart, longer than the four MMAs of a 64-token k-step take.
+template <int BN, int NI>
 struct TileTA {
-    static constexpr int A_COL = BN;
-    static constexpr int TMEM_COLS = BN + STAGES * A_COLS <= 256 ? 256 : 512;  // a power of two
+    static constexpr int A_COL = BN * NI;
+    static constexpr int TMEM_COLS = A_COL + STAGES * A_COLS <= 256 ? 256 : 512;  // a power of two
+    static constexpr int THREADS = 32 * (6 + NI - 1);  // issuers past the first are warps 6, 7, ...
     static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * Tile<BN>::B_STAGE + 256;
+    static_assert(A_COL + STAGES * A_COLS <= 512, "accumulators and A stages exceed tensor memory");
 };
+constexpr int TA_ISSUERS = 2;
 
 // Expand 16 sign bits (bit i = element i of a k-run) into 8 bf16x2 words:
 // word i holds elements (2i, 2i+1) as +1.0 (0x3F80) or -1.0 (0xBF80).
@@ -251,12 +257,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
-template <int BN>
-__global__ void __launch_bounds__(THREADS, 1)
+template <int BN, int NI>
+__global__ void __launch_bounds__(TileTA<BN, NI>::THREADS, 1)
     gemm_kernel_ta(const __grid_constant__ CUtensorMap tmap_u, const uint32_t* __restrict__ packed,
                 const float* __restrict__ s, int out, int K, int tokens, float* __restrict__ o,
                 unsigned* status) {
-    constexpr int B_STAGE = Tile<BN>::B_STAGE, TMEM_COLS = TileTA<BN>::TMEM_COLS, A_COL = TileTA<BN>::A_COL;
+    constexpr int B_STAGE = Tile<BN>::B_STAGE, TMEM_COLS = TileTA<BN, NI>::TMEM_COLS, A_COL = TileTA<BN, NI>::A_COL;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned for the 128-byte swizzle; offsetting the array itself
     // keeps derived pointers in the shared address space
@@ -282,7 +288,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(full0 + 8 * st, 1 + UNPACK_THREADS);
             mbar_init(empty0 + 8 * st, 1);
         }
-        mbar_init(accf, 1);
+        mbar_init(accf, NI);  // one commit per issuer
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tensormap(&tmap_u);
@@ -313,10 +319,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
                 mbar_wait(full0 + 8 * (kb % STAGES), (kb / STAGES) & 1, status);
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp >= 6) {
+        // issuer `isr` takes k-steps isr, isr + NI, ... into accumulator columns [isr BN, (isr + 1) BN)
+        const int isr = warp == 1 ? 0 : warp - 5;
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(BM, BN);
-            for (int kb = 0; kb < nkb; ++kb) {
+            const uint32_t idesc = idesc_bf16_f32(BM, BN), acc = tmem + isr * BN;
+            for (int kb = isr; kb < nkb; kb += NI) {
                 const int st = kb % STAGES, round = kb / STAGES;
                 if (!mbar_wait(full0 + 8 * st, round & 1, status)) {
                     *abort_flag = 1;
@@ -326,10 +334,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t a_tmem = tmem + A_COL + st * A_COLS, b_base = smem_addr(sB + st * B_STAGE);
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)  // 16 k = 8 TMEM columns of A, 32 bytes of a B row
-                    umma_f16_tmem_a(tmem, a_tmem + kk * 8, smem_desc_sw128(b_base + kk * 32), idesc, (kb | kk) != 0);
+                    umma_f16_tmem_a(acc, a_tmem + kk * 8, smem_desc_sw128(b_base + kk * 32), idesc,
+                                    kb != isr || kk != 0);
                 umma_commit(empty0 + 8 * st);
             }
-            umma_commit(accf);  // fires once every issued MMA has completed
+            umma_commit(accf);  // fires once every MMA this thread issued has completed
         }
     } else {
         // ---- unpack: thread `row` writes row `row` of every A stage into TMEM
@@ -414,17 +423,28 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];
+                float acc[32];
                 tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + c0, v);
                 tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(v[j]);
+                // the issuers' sums, added in issuer order (an issuer without k-steps wrote nothing)
+#pragma unroll 1
+                for (int i = 1; i < NI && i < nkb; ++i) {
+                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + i * BN + c0, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) acc[j] += __uint_as_float(v[j]);
+                }
                 if (m < out) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int n = n0 + c0 + j;
                         if (n < tokens) {
                             if (split)
-                                atomicAdd(o + (long long)n * out + m, sr * __uint_as_float(v[j]));
+                                atomicAdd(o + (long long)n * out + m, sr * acc[j]);
                             else
-                                o[(long long)n * out + m] = sr * __uint_as_float(v[j]);
+                                o[(long long)n * out + m] = sr * acc[j];
                         }
                     }
                 }
@@ -475,8 +495,15 @@ cudaError_t launch_tile(const uint32_t* packed, const float* s, int out, int K, 
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     // 64-token tiles: A stages in TMEM; wider tiles: A stages in shared memory
     constexpr bool kTA = BN <= 64;
-    auto kern = kTA ? gemm_kernel_ta<BN> : gemm_kernel<BN>;
-    constexpr size_t smem = kTA ? TileTA<BN>::SMEM_BYTES : Tile<BN>::SMEM_BYTES;
+    using TA = TileTA<kTA ? BN : 64, TA_ISSUERS>;
+    auto kern = [] {
+        if constexpr (kTA)
+            return gemm_kernel_ta<BN, TA_ISSUERS>;
+        else
+            return gemm_kernel<BN>;
+    }();
+    constexpr size_t smem = kTA ? TA::SMEM_BYTES : Tile<BN>::SMEM_BYTES;
+    constexpr int threads = kTA ? TA::THREADS : THREADS;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -492,7 +519,7 @@ cudaError_t launch_tile(const uint32_t* packed, const float* s, int out, int K, 
         cudaError_t e = cudaMemsetAsync(o, 0, (size_t)tokens * out * sizeof(float), st);
         if (e != cudaSuccess) return e;
     }
-    kern<<<grid, THREADS, smem, st>>>(map, packed, s, out, K, tokens, o, status);
+    kern<<<grid, threads, smem, st>>>(map, packed, s, out, K, tokens, o, status);
     return cudaGetLastError();
 }
 
