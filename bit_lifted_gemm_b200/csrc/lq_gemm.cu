@@ -51,15 +51,16 @@ struct Tile {
 // Its k-steps alternate between NI issuing threads in separate warps, each with
 // an accumulator of its own: one thread's commits complete one after another,
 // ~400 clocks apart, longer than the four MMAs of a 64-token k-step take.
-template <int BN, int NI>
+template <int BN, int NI, int S>
 struct TileTA {
     static constexpr int A_COL = BN * NI;
-    static constexpr int TMEM_COLS = A_COL + STAGES * A_COLS <= 256 ? 256 : 512;  // a power of two
+    static constexpr int TMEM_COLS = A_COL + S * A_COLS <= 256 ? 256 : 512;  // a power of two
     static constexpr int THREADS = 32 * (6 + NI - 1);  // issuers past the first are warps 6, 7, ...
-    static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * Tile<BN>::B_STAGE + 256;
-    static_assert(A_COL + STAGES * A_COLS <= 512, "accumulators and A stages exceed tensor memory");
+    static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + S * Tile<BN>::B_STAGE + 256;
+    static_assert(A_COL + S * A_COLS <= 512, "accumulators and A stages exceed tensor memory");
 };
-constexpr int TA_ISSUERS = 2;
+constexpr int TA_ISSUERS = 2, TA_STAGES = 4;
+constexpr bool TA_EAGER = false, TA_SPLIT = true;
 
 // Expand 16 sign bits (bit i = element i of a k-run) into 8 bf16x2 words:
 // word i holds elements (2i, 2i+1) as +1.0 (0x3F80) or -1.0 (0xBF80).
@@ -76,11 +77,85 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
+// Epilogue of both kernels, run by the four warps that own the TMEM lane
+// quarters (warp & 3): o[t][r] = s[r] * (sum of the nacc accumulators, columns
+// acc_stride apart, added in order) for the 128 x BN tile at (m0, n0). With a
+// tensor map for o the warps stage the tile in shared memory ([BN][128] fp32,
+// in the operand stages, idle once the accumulators are final) and one thread
+// writes it with one TMA store, or with a TMA add when K is split (two addends
+// into a zeroed o: the same sum in either order); rows and tokens past the
+// tensor are clipped. Without one (o rows not 16-byte aligned) every thread
+// stores its row. `done` is this thread's wait on the accumulators; whether to
+// go on is decided once for all four warps, so the named barriers are reached
+// by all of them or none.
+template <int BN>
+__device__ __forceinline__ void epilogue_tile(uint32_t tmem, int nacc, int acc_stride, bool done,
+                                              const CUtensorMap* omap, bool tma_out, bool split, float* stage,
+                                              volatile int* abort_flag, volatile int* go_word, const float* s,
+                                              float* o, int out, int tokens, int m0, int n0, int warp, int lane) {
+    if (!done) *abort_flag = 1;
+    __syncwarp();
+    named_bar_sync(1, 128);
+    if (warp == 2 && lane == 0) *go_word = *abort_flag ? 0 : 1;
+    named_bar_sync(1, 128);
+    if (!*go_word) return;
+    tc_fence_after();
+    const int q = warp & 3;  // this warp's TMEM lane quadrant
+    const int m = m0 + q * 32 + lane;
+    const float sr = m < out ? __ldg(s + m) : 0.f;
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        float acc[32];
+        tmem_ld_32x32b_x32(lane_base + c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(v[j]);
+#pragma unroll 1
+        for (int i = 1; i < nacc; ++i) {
+            tmem_ld_32x32b_x32(lane_base + i * acc_stride + c0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[j] += __uint_as_float(v[j]);
+        }
+        if (tma_out) {
+            // token row c0 + j of the box, this lane's row of W_q at q * 32 + lane:
+            // a warp writes 128 consecutive bytes per token
+#pragma unroll
+            for (int j = 0; j < 32; ++j) stage[(c0 + j) * BM + q * 32 + lane] = sr * acc[j];
+        } else if (m < out) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int n = n0 + c0 + j;
+                if (n < tokens) {
+                    if (split)
+                        atomicAdd(o + (long long)n * out + m, sr * acc[j]);
+                    else
+                        o[(long long)n * out + m] = sr * acc[j];
+                }
+            }
+        }
+    }
+    if (tma_out) {
+        fence_proxy_async_smem();  // the staged tile, visible to the bulk copy
+        named_bar_sync(1, 128);
+        if (warp == 2 && lane == 0) {
+            if (split)
+                tma_reduce_add_2d(omap, smem_addr(stage), m0, n0);
+            else
+                tma_store_2d(omap, smem_addr(stage), m0, n0);
+            bulk_commit_group();
+            bulk_wait_group_all();  // complete before the CTA exits and its shared memory is reused
+        }
+    }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmap_u, const uint32_t* __restrict__ packed,
-                const float* __restrict__ s, int out, int K, int tokens, float* __restrict__ o,
-                unsigned* status) {
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_u, const __grid_constant__ CUtensorMap tmap_o,
+                const uint32_t* __restrict__ packed, const float* __restrict__ s, int out, int K, int tokens,
+                float* __restrict__ o, int tma_out, unsigned* status) {
     constexpr int B_STAGE = Tile<BN>::B_STAGE, TMEM_COLS = Tile<BN>::TMEM_COLS;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned for the 128-byte swizzle; offsetting the array itself
@@ -91,6 +166,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* go_word = reinterpret_cast<volatile int*>(tmem_slot + 2);
     const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + STAGES), accf = smem_addr(bars + 2 * STAGES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -217,33 +293,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int q = 0; q < 16; ++q) cur[q] = nxt[q];
         }
 
-        // ---- epilogue: TMEM -> registers -> s[r] * acc -> o[t][r]
+        // ---- epilogue: TMEM -> registers -> s[r] * acc -> o[t][r], staged in the A / B stages
+        static_assert(STAGES * (A_STAGE + B_STAGE) >= BN * BM * 4, "the output tile must fit the operand stages");
         const bool done = mbar_wait(accf, 0, status);
-        tc_fence_after();
-        // tcgen05.ld is warp-collective: decide for the whole warp at once
-        if (__all_sync(0xffffffffu, done && !*abort_flag)) {
-            const int q = warp & 3;  // this warp's TMEM lane quadrant
-            const int m = m0 + q * 32 + lane;
-            const float sr = m < out ? __ldg(s + m) : 0.f;
-#pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + c0, v);
-                tmem_ld_wait();
-                if (m < out) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int n = n0 + c0 + j;
-                        if (n < tokens) {
-                            if (split)
-                                atomicAdd(o + (long long)n * out + m, sr * __uint_as_float(v[j]));
-                            else
-                                o[(long long)n * out + m] = sr * __uint_as_float(v[j]);
-                        }
-                    }
-                }
-            }
-        }
+        epilogue_tile<BN>(tmem, 1, 0, done, &tmap_o, tma_out != 0, split, reinterpret_cast<float*>(sA), abort_flag,
+                          go_word, s, o, out, tokens, m0, n0, warp, lane);
     }
 
     // lane 0 of the producer and issuer warps ran its role alone: reconverge
@@ -257,12 +311,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
-template <int BN, int NI>
-__global__ void __launch_bounds__(TileTA<BN, NI>::THREADS, 1)
-    gemm_kernel_ta(const __grid_constant__ CUtensorMap tmap_u, const uint32_t* __restrict__ packed,
-                const float* __restrict__ s, int out, int K, int tokens, float* __restrict__ o,
-                unsigned* status) {
-    constexpr int B_STAGE = Tile<BN>::B_STAGE, TMEM_COLS = TileTA<BN, NI>::TMEM_COLS, A_COL = TileTA<BN, NI>::A_COL;
+template <int BN, int NI, int S>
+__global__ void __launch_bounds__(TileTA<BN, NI, S>::THREADS, 1)
+    gemm_kernel_ta(const __grid_constant__ CUtensorMap tmap_u, const __grid_constant__ CUtensorMap tmap_o,
+                const uint32_t* __restrict__ packed, const float* __restrict__ s, int out, int K, int tokens,
+                float* __restrict__ o, int tma_out, unsigned* status) {
+    constexpr int STAGES = S;  // A stages in TMEM, B stages in shared memory
+    constexpr int B_STAGE = Tile<BN>::B_STAGE, TMEM_COLS = TileTA<BN, NI, S>::TMEM_COLS, A_COL = TileTA<BN, NI, S>::A_COL;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned for the 128-byte swizzle; offsetting the array itself
     // keeps derived pointers in the shared address space
@@ -271,6 +326,7 @@ __global__ void __launch_bounds__(TileTA<BN, NI>::THREADS, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* go_word = reinterpret_cast<volatile int*>(tmem_slot + 2);
     const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + STAGES), accf = smem_addr(bars + 2 * STAGES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -402,6 +458,12 @@ __global__ void __launch_bounds__(TileTA<BN, NI>::THREADS, 1)
                 // word j holds k-elements (2j, 2j+1): TMEM column j of the stage
                 tmem_st_32x32b_x32(a_lane + st * A_COLS, v);
                 pending = st;
+                if (TA_EAGER) {
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(full0 + 8 * st);
+                    pending = -1;
+                }
             }
 #pragma unroll
             for (int q = 0; q < 16; ++q) cur[q] = nxt[q];
@@ -412,44 +474,12 @@ __global__ void __launch_bounds__(TileTA<BN, NI>::THREADS, 1)
             mbar_arrive(full0 + 8 * pending);
         }
 
-        // ---- epilogue: TMEM -> registers -> s[r] * acc -> o[t][r]
+        // ---- epilogue: TMEM -> registers -> s[r] * acc -> o[t][r], staged in the B stages; the
+        // issuers' sums are added in issuer order (an issuer without k-steps wrote nothing)
+        static_assert(STAGES * B_STAGE >= BN * BM * 4, "the output tile must fit the B stages");
         const bool done = mbar_wait(accf, 0, status);
-        tc_fence_after();
-        // tcgen05.ld is warp-collective: decide for the whole warp at once
-        if (__all_sync(0xffffffffu, done && !*abort_flag)) {
-            const int q = warp & 3;  // this warp's TMEM lane quadrant
-            const int m = m0 + q * 32 + lane;
-            const float sr = m < out ? __ldg(s + m) : 0.f;
-#pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                uint32_t v[32];
-                float acc[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + c0, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(v[j]);
-                // the issuers' sums, added in issuer order (an issuer without k-steps wrote nothing)
-#pragma unroll 1
-                for (int i = 1; i < NI && i < nkb; ++i) {
-                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + i * BN + c0, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) acc[j] += __uint_as_float(v[j]);
-                }
-                if (m < out) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int n = n0 + c0 + j;
-                        if (n < tokens) {
-                            if (split)
-                                atomicAdd(o + (long long)n * out + m, sr * acc[j]);
-                            else
-                                o[(long long)n * out + m] = sr * acc[j];
-                        }
-                    }
-                }
-            }
-        }
+        epilogue_tile<BN>(tmem, NI < nkb ? NI : nkb, BN, done, &tmap_o, tma_out != 0, split,
+                          reinterpret_cast<float*>(sB), abort_flag, go_word, s, o, out, tokens, m0, n0, warp, lane);
     }
 
     // lane 0 of the producer and issuer warps ran its role alone: reconverge
@@ -493,12 +523,24 @@ cudaError_t launch_tile(const uint32_t* packed, const float* s, int out, int K, 
                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    // o [tokens][out] fp32 for the TMA-store epilogue: rows must be 16-byte aligned
+    CUtensorMap omap;
+    int tma_out = 0;
+    if (out % 4 == 0 && (reinterpret_cast<uintptr_t>(o) & 15u) == 0) {
+        cuuint64_t odim[2] = {(cuuint64_t)out, (cuuint64_t)tokens};
+        cuuint64_t ostride[1] = {(cuuint64_t)out * 4};
+        cuuint32_t obox[2] = {BM, BN};
+        tma_out = encode(&omap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, o, odim, ostride, obox, estride,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
+    if (!tma_out) omap = map;  // unused by the kernel
     // 64-token tiles: A stages in TMEM; wider tiles: A stages in shared memory
     constexpr bool kTA = BN <= 64;
-    using TA = TileTA<kTA ? BN : 64, TA_ISSUERS>;
+    using TA = TileTA<kTA ? BN : 64, TA_ISSUERS, TA_STAGES>;
     auto kern = [] {
         if constexpr (kTA)
-            return gemm_kernel_ta<BN, TA_ISSUERS>;
+            return gemm_kernel_ta<BN, TA_ISSUERS, TA_STAGES>;
         else
             return gemm_kernel<BN>;
     }();
@@ -514,12 +556,12 @@ cudaError_t launch_tile(const uint32_t* packed, const float* s, int out, int K, 
     }
     dim3 grid((out + BM - 1) / BM, (tokens + BN - 1) / BN, 1);
     const int nkb = (K + BK - 1) / BK;
-    if ((long long)grid.x * grid.y < num_sms && nkb >= 16) {  // too few tiles for the SMs: split K in two
+    if ((!kTA || TA_SPLIT) && (long long)grid.x * grid.y < num_sms && nkb >= 16) {  // too few tiles for the SMs: split K in two
         grid.z = 2;
         cudaError_t e = cudaMemsetAsync(o, 0, (size_t)tokens * out * sizeof(float), st);
         if (e != cudaSuccess) return e;
     }
-    kern<<<grid, threads, smem, st>>>(map, packed, s, out, K, tokens, o, status);
+    kern<<<grid, threads, smem, st>>>(map, omap, packed, s, out, K, tokens, o, tma_out, status);
     return cudaGetLastError();
 }
 
