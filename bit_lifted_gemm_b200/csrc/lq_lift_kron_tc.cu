@@ -13,9 +13,11 @@
 // kron_z_kernel: M = 128 tokens, N = n2 (the j2 of one i1), K = i2 (padded to a
 // multiple of 64; the padded positions of B are zero). A = the bf16 activations
 // themselves, by TMA (128-byte swizzle); B = r1-scaled rows of Q2, which are
-// fp32: split on the fly into three bf16 parts (hi, mid, lo: 24 significant
-// bits), each a B operand accumulating into the same fp32 TMEM tile. Four i1
-// per CTA, one accumulator each. Z leaves in fp32.
+// fp32: split into three bf16 parts (hi, mid, lo: 24 significant bits), each a
+// B operand accumulating into the same fp32 TMEM tile. One i1 per CTA, whose B
+// parts are built once and kept while the CTA runs through its range of token
+// tiles (grid: n1 x ranges); two TMEM accumulators, so the epilogue of one tile
+// overlaps the MMAs of the next. Z leaves in fp32 by TMA store.
 //
 // kron_y_kernel: per token, M = j1 (Q1 rows, padded to 128 with zero rows),
 // N = j2, K = i1 (n1 <= 64: one 64-wide atom). A = Q1 in three bf16 parts
