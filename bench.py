@@ -454,13 +454,13 @@ def bench_kron(torch, lq, l2, reps=50):
 
 
 def bench_encode(torch, lq):
-    """Encoder (offline): seconds per million weights for LQ-24/10, LQ-16/8 and
-    LQ-32/16 on seeded Gaussian weights and projections, each sample sized to a
-    second or two (the cost per block grows as 2^(D-d))."""
+    """Encoder (offline): seconds per million weights for LQ-24/10, LQ-16/8,
+    LQ-32/16 and LQ-32/20 on seeded Gaussian weights and projections, each sample
+    sized to a second or less (the cost per block grows as 2^(D-d))."""
     dev = torch.device("cuda")
     res = {}
     for name, d, D, rows, in_dim in (("lq24_10", 10, 24, 26, 5120), ("lq16_8", 8, 16, 256, 4096),
-                                     ("lq32_16", 16, 32, 32, 4096)):
+                                     ("lq32_16", 16, 32, 32, 4096), ("lq32_20", 20, 32, 256, 4000)):
         g = np.random.default_rng(0x4C51 + D)
         M = torch.from_numpy((g.standard_normal((d, D)) / np.sqrt(D)).astype(np.float32)).to(dev)
         w = torch.from_numpy(g.standard_normal((rows, in_dim)).astype(np.float32)).to(dev)

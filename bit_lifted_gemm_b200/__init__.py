@@ -18,15 +18,19 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liblq.so")
+# LQ_DEBUG=1 selects the debug build (device-side bounds checks, LQ_ERR_BOUNDS)
+DEBUG = os.environ.get("LQ_DEBUG", "") not in ("", "0")
+LIB_PATH = os.path.join(_HERE, "liblq_debug.so" if DEBUG else "liblq.so")
 
 LQ_OK, LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_TIMEOUT, LQ_ERR_TOO_LARGE = 0, 1, 2, 3, 4, 5
+LQ_ERR_BOUNDS = 6
 LQ_F32, LQ_BF16 = 0, 1
 GEMV_NOALLOC_SCRATCH_BYTES = 4 << 20  # LQ_GEMV_NOALLOC_SCRATCH_BYTES of include/lq.h
 
 SYMBOLS = ("lq_status_str", "lq_lifted_dim", "lq_pack_signs", "lq_unpack_signs", "lq_lift_activations",
            "lq_lift_activations_kron", "lq_gemv_workspace_size", "lq_gemv", "lq_gemv_noalloc", "lq_lift_gemv",
-           "lq_gemm", "lq_encode", "lq_selftest_wait_timeout", "lq_get_device_status")
+           "lq_gemm", "lq_encode", "lq_selftest_wait_timeout", "lq_selftest_bounds", "lq_is_debug_build",
+           "lq_get_device_status")
 
 
 class LQError(RuntimeError):
@@ -37,7 +41,8 @@ class LQError(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"liblq.so not built at {LIB_PATH}; run `python bit_lifted_gemm_b200/build.py`")
+        how = "python bit_lifted_gemm_b200/build.py" + (" --debug" if DEBUG else "")
+        raise ImportError(f"{os.path.basename(LIB_PATH)} not built at {LIB_PATH}; run `{how}`")
     lib = ctypes.CDLL(LIB_PATH)
     p, i = ctypes.c_void_p, ctypes.c_int
     lib.lq_status_str.restype = ctypes.c_char_p
@@ -65,6 +70,10 @@ def _load() -> ctypes.CDLL:
     lib.lq_encode.restype = i
     lib.lq_selftest_wait_timeout.restype = i
     lib.lq_selftest_wait_timeout.argtypes = [ctypes.c_uint, p]
+    lib.lq_selftest_bounds.restype = i
+    lib.lq_selftest_bounds.argtypes = [p]
+    lib.lq_is_debug_build.restype = i
+    lib.lq_is_debug_build.argtypes = []
     lib.lq_encode.argtypes = [p, i, i, p, i, i, p, i, p, p]
     lib.lq_gemm.argtypes = [p, p, i, i, p, i, p, p]
     lib.lq_get_device_status.restype = i

@@ -1,8 +1,12 @@
 """Build liblq.so (the C-ABI library of sm_100a kernels) in-tree with nvcc.
 
-    python bit_lifted_gemm_b200/build.py [--force] [--verbose-ptxas]
+    python bit_lifted_gemm_b200/build.py [--force] [--verbose-ptxas] [--debug]
 
-(Run it by path: importing the package loads liblq.so.)
+--debug builds liblq_debug.so instead: the same sources with -DLQ_DEBUG, whose
+kernels check the element index of each computed global access against its
+buffer and report LQ_ERR_BOUNDS instead of touching memory out of bounds. The
+package loads it when the environment has LQ_DEBUG=1.
+(Run it by path: importing the package loads the library.)
 """
 
 from __future__ import annotations
@@ -18,6 +22,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblq.so")
 OBJDIR = os.path.join(PKG, "_build")
+LIB_DEBUG = os.path.join(PKG, "liblq_debug.so")
+OBJDIR_DEBUG = os.path.join(PKG, "_build_debug")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -41,25 +47,28 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
-    os.makedirs(OBJDIR, exist_ok=True)
+def build(force: bool = False, ptxas_verbose: bool = False, debug: bool = False) -> str:
+    objdir, lib = (OBJDIR_DEBUG, LIB_DEBUG) if debug else (OBJDIR, LIB)
+    flags = FLAGS + (["-DLQ_DEBUG"] if debug else [])
+    os.makedirs(objdir, exist_ok=True)
     headers = _headers()
     objs = []
     for src in _sources():
-        obj = os.path.join(OBJDIR, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or ptxas_verbose or _stale(obj, [src] + headers):
-            cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+            cmd = [NVCC, *ARCH, *flags, "-c", src, "-o", obj]
             if ptxas_verbose:
                 cmd += ["-Xptxas", "-v"]
             subprocess.check_call(cmd)
-    if force or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lrt",
                                "-lpthread"])
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, ptxas_verbose="--verbose-ptxas" in sys.argv))
+    print(build(force="--force" in sys.argv, ptxas_verbose="--verbose-ptxas" in sys.argv,
+                debug="--debug" in sys.argv))

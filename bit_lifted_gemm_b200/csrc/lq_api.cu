@@ -134,6 +134,7 @@ const char* lq_status_str(int status) {
         case LQ_ERR_CUDA: return "LQ_ERR_CUDA";
         case LQ_ERR_TIMEOUT: return "LQ_ERR_TIMEOUT";
         case LQ_ERR_TOO_LARGE: return "LQ_ERR_TOO_LARGE";
+        case LQ_ERR_BOUNDS: return "LQ_ERR_BOUNDS";
         default: return "LQ_ERR_UNKNOWN";
     }
 }
@@ -217,7 +218,7 @@ int lq_encode(const float* w, int rows, int in, const float* M, int d, int D, ui
               void* stream) {
     if (!w || !M || !packed || !aligned16(w) || !aligned16(M) || !aligned16(packed)) return LQ_ERR_INVALID_ARG;
     if (err && !aligned16(err)) return LQ_ERR_INVALID_ARG;
-    if (rows < 1 || in < 1 || d < 1 || d > 16 || D < d || D > 63 || D - d > 24 || in % d != 0)
+    if (rows < 1 || in < 1 || d < 1 || d > 24 || D < d || D > 63 || D - d > 24 || in % d != 0)
         return LQ_ERR_INVALID_ARG;
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
@@ -323,7 +324,35 @@ int lq_get_device_status(void* stream) {
     if (cudaMemcpyFromSymbolAsync(&v, g_lq_status_read, sizeof(v), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return LQ_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return LQ_ERR_CUDA;
+#ifdef LQ_DEBUG
+    // every file's flag is read and cleared, whichever is set
+    const unsigned bounds = lq::debug_take_gemm() | lq::debug_take_lift() | lq::debug_take_lift_kron() |
+                            lq::debug_take_lift_tc() | lq::debug_take_lift_kron_tc() | lq::debug_take_encode() |
+                            lq::debug_take_pack() | lq::debug_take_selftest();
+    if (bounds) return LQ_ERR_BOUNDS;
+#endif
     return (v & LQ_DEV_TIMEOUT) ? LQ_ERR_TIMEOUT : LQ_OK;
+}
+
+int lq_selftest_bounds(void* stream) {
+#ifdef LQ_DEBUG
+    if (fault_is("launch")) return LQ_ERR_CUDA;
+    const int sm = is_sm100();
+    if (sm < 0) return LQ_ERR_CUDA;
+    if (sm == 0) return LQ_ERR_UNSUPPORTED;
+    return from_cuda(lq::launch_selftest_bounds(static_cast<cudaStream_t>(stream)));
+#else
+    (void)stream;
+    return LQ_ERR_UNSUPPORTED;
+#endif
+}
+
+int lq_is_debug_build(void) {
+#ifdef LQ_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
 }
 
 // ---------------------------------------------------------------- decode GEMV without allocation

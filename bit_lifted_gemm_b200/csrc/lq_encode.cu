@@ -24,6 +24,7 @@
 
 #include <algorithm>
 
+#include "lq_debug.cuh"
 #include "lq_internal.h"
 
 namespace lq {
@@ -312,18 +313,21 @@ __global__ void __launch_bounds__(EN_THREADS, 1) encode_kernel(const EncArgs p) 
         const int row = (int)(u / p.nblk), b = (int)(u - (long long)row * p.nblk);
         uint64_t y = 0;
         double e = __longlong_as_double(0x7ff8000000000000ll);  // NaN: singular M M^T or M_B
-        if (!singular) encode_block<MAXD>(Md, P, Bi, G, d, D, p.w + (long long)row * p.in + (long long)b * d, lane, y, e);
+        const bool w_ok = LQ_IN_BOUNDS((long long)row * p.in + (long long)b * d + d - 1, (long long)p.rows * p.in);
+        if (!singular && w_ok)
+            encode_block<MAXD>(Md, P, Bi, G, d, D, p.w + (long long)row * p.in + (long long)b * d, lane, y, e);
         if (lane == 0) {
-            if (p.err) p.err[u] = (float)e;
+            if (p.err && LQ_IN_BOUNDS(u, units)) p.err[u] = (float)e;
             // bits [b D, b D + D) of the row: words q, q + 1 and (past 64 bits) q + 2
             uint32_t* words = p.packed + (long long)row * nq;
             const long long bit0 = (long long)b * D;
             const int q = (int)(bit0 >> 5), o = (int)(bit0 & 31);
             const uint64_t sh = y << o;
             const uint32_t w0 = (uint32_t)sh, w1 = (uint32_t)(sh >> 32), w2 = o ? (uint32_t)(y >> (64 - o)) : 0u;
-            if (w0) atomicOr(words + q, w0);
-            if (w1) atomicOr(words + q + 1, w1);
-            if (w2) atomicOr(words + q + 2, w2);
+            // every word a block touches lies within its own row (K / 32 words)
+            if (w0 && LQ_IN_BOUNDS(q, nq)) atomicOr(words + q, w0);
+            if (w1 && LQ_IN_BOUNDS(q + 1, nq)) atomicOr(words + q + 1, w1);
+            if (w2 && LQ_IN_BOUNDS(q + 2, nq)) atomicOr(words + q + 2, w2);
         }
     }
 }
@@ -371,7 +375,10 @@ cudaError_t launch_encode(const float* w, int rows, int in, const float* M, int 
     if (d <= 8) return launch_encode_t<8>(p, smem, st);
     if (d <= 10) return launch_encode_t<10>(p, smem, st);
     if (d <= 12) return launch_encode_t<12>(p, smem, st);
-    return launch_encode_t<16>(p, smem, st);
+    if (d <= 16) return launch_encode_t<16>(p, smem, st);
+    return launch_encode_t<24>(p, smem, st);
 }
 
 }  // namespace lq
+
+LQ_DEBUG_FLAG_TAKE(debug_take_encode)

@@ -26,6 +26,7 @@
 // stores into the async proxy before arriving. Every wait is bounded.
 #include <cuda.h>
 
+#include "lq_debug.cuh"
 #include "lq_internal.h"
 #include "lq_sm100.cuh"
 
@@ -125,7 +126,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tmem, int nacc, int acc_s
     tc_fence_after();
     const int q = warp & 3;  // this warp's TMEM lane quadrant
     const int m = m0 + q * 32 + lane;
-    const float sr = m < out ? __ldg(s + m) : 0.f;
+    const float sr = m < out && LQ_IN_BOUNDS(m, out) ? __ldg(s + m) : 0.f;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
     for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -151,7 +152,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tmem, int nacc, int acc_s
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int n = n0 + c0 + j;
-                if (n < tokens) {
+                if (n < tokens && LQ_IN_BOUNDS((long long)n * out + m, (long long)tokens * out)) {
                     if (split)
                         atomicAdd(o + (long long)n * out + m, sr * acc[j]);
                     else
@@ -270,7 +271,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         // do not wait a memory round trip per k-step.
         const bool vec = (kw & 3) == 0;  // 16-byte aligned rows
         auto load16 = [&](int kg0, uint32_t (&w)[16]) {
-            if (vec && (kg0 & 1) == 0 && 2 * kg0 + 16 <= kw) {
+            if (vec && (kg0 & 1) == 0 && 2 * kg0 + 16 <= kw &&
+                LQ_IN_BOUNDS((long long)grow * kw + 2 * kg0 + 15, (long long)out * kw)) {
                 const uint4* src = reinterpret_cast<const uint4*>(prow + 2 * kg0);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -282,7 +284,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             } else {
 #pragma unroll
-                for (int q = 0; q < 16; ++q) w[q] = 2 * kg0 + q < kw ? __ldg(prow + 2 * kg0 + q) : 0u;  // u is zero past K
+                for (int q = 0; q < 16; ++q)  // u is zero past K
+                    w[q] = 2 * kg0 + q < kw && LQ_IN_BOUNDS((long long)grow * kw + 2 * kg0 + q, (long long)out * kw)
+                               ? __ldg(prow + 2 * kg0 + q)
+                               : 0u;
             }
         };
         uint32_t cur[16], nxt[16];
@@ -432,7 +437,8 @@ __global__ void __launch_bounds__(TileTA<BN, NI, S>::THREADS, 1)
         // do not wait a memory round trip per k-step.
         const bool vec = (kw & 3) == 0;  // 16-byte aligned rows
         auto load16 = [&](int kg0, uint32_t (&w)[16]) {
-            if (vec && (kg0 & 1) == 0 && 2 * kg0 + 16 <= kw) {
+            if (vec && (kg0 & 1) == 0 && 2 * kg0 + 16 <= kw &&
+                LQ_IN_BOUNDS((long long)grow * kw + 2 * kg0 + 15, (long long)out * kw)) {
                 const uint4* src = reinterpret_cast<const uint4*>(prow + 2 * kg0);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -444,7 +450,10 @@ __global__ void __launch_bounds__(TileTA<BN, NI, S>::THREADS, 1)
                 }
             } else {
 #pragma unroll
-                for (int q = 0; q < 16; ++q) w[q] = 2 * kg0 + q < kw ? __ldg(prow + 2 * kg0 + q) : 0u;  // u is zero past K
+                for (int q = 0; q < 16; ++q)  // u is zero past K
+                    w[q] = 2 * kg0 + q < kw && LQ_IN_BOUNDS((long long)grow * kw + 2 * kg0 + q, (long long)out * kw)
+                               ? __ldg(prow + 2 * kg0 + q)
+                               : 0u;
             }
         };
         uint32_t cur[16], nxt[16];
@@ -601,3 +610,5 @@ cudaError_t launch_gemm(const uint32_t* packed, const float* s, int out, int K, 
 }
 
 }  // namespace lq
+
+LQ_DEBUG_FLAG_TAKE(debug_take_gemm)

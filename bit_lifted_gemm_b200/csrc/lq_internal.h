@@ -52,6 +52,21 @@ cudaError_t launch_encode(const float* w, int rows, int in, const float* M, int 
 
 // Self-test of the bounded waits: one wait that nothing completes, limit_us long.
 cudaError_t launch_selftest_wait_timeout(unsigned limit_us, unsigned* status, cudaStream_t st);
+// Debug build: one failed bounds check with no access behind it (cudaErrorNotSupported in release).
+cudaError_t launch_selftest_bounds(cudaStream_t st);
+
+#ifdef LQ_DEBUG
+// Debug build: read and clear the bounds flag of each source file (non-zero after
+// a failed check), on the current device.
+unsigned debug_take_gemm();
+unsigned debug_take_lift();
+unsigned debug_take_lift_kron();
+unsigned debug_take_lift_tc();
+unsigned debug_take_lift_kron_tc();
+unsigned debug_take_encode();
+unsigned debug_take_pack();
+unsigned debug_take_selftest();
+#endif
 
 // Decode GEMV (lq_decode.h): the quantizer writes u's digit planes into the
 // caller's workspace, then the mma.sync kernel (batch 1..2, or when the

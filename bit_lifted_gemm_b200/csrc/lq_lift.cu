@@ -74,7 +74,7 @@ __device__ __forceinline__ void lift_and_store(const LiftArgs& p, const Range& r
 #pragma unroll
         for (int q = 0; q < TT; ++q) {
             int t = tg * TT + q;
-            if (t < nt) store_u(p.u, p.u_bf16, (long long)(t0 + t) * p.K + kk, acc[q]);
+            if (t < nt) store_u(p.u, p.u_bf16, (long long)(t0 + t) * p.K + kk, (long long)p.batch * p.K, acc[q]);
         }
     }
     if (blockIdx.x == gridDim.x - 1) {
@@ -82,7 +82,7 @@ __device__ __forceinline__ void lift_and_store(const LiftArgs& p, const Range& r
         const int npad = p.K - kreal;
         for (int item = threadIdx.x; item < npad * nt; item += blockDim.x) {
             int t = item / npad, k = kreal + item % npad;
-            store_u(p.u, p.u_bf16, (long long)(t0 + t) * p.K + k, 0.f);
+            store_u(p.u, p.u_bf16, (long long)(t0 + t) * p.K + k, (long long)p.batch * p.K, 0.f);
         }
     }
 }
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(256) lift_decode_kernel(LiftArgs p) {
     for (int i = threadIdx.x; i < p.d * p.D; i += blockDim.x) Ms[i] = __ldg(p.M + i);
     for (int i = threadIdx.x; i < span * nt; i += blockDim.x) {
         int t = i / span, j = i - t * span;
-        as[t * span + j] = load_act(p.a, p.a_bf16, (long long)(t0 + t) * p.in + r.lo + j);
+        as[t * span + j] = load_act(p.a, p.a_bf16, (long long)(t0 + t) * p.in + r.lo + j, (long long)p.batch * p.in);
     }
     __syncthreads();
 
@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(256) lift_prefill_kernel(LiftArgs p) {
     for (int i = threadIdx.x; i < p.d * p.D; i += blockDim.x) Ms[i] = __ldg(p.M + i);
     for (int i = threadIdx.x; i < span * PRE_TB; i += blockDim.x) {
         int t = i / span, j = i - t * span;
-        as[j * PRE_TB + t] = t < nt ? load_act(p.a, p.a_bf16, (long long)(t0 + t) * p.in + r.lo + j) : 0.f;
+        as[j * PRE_TB + t] = t < nt ? load_act(p.a, p.a_bf16, (long long)(t0 + t) * p.in + r.lo + j, (long long)p.batch * p.in) : 0.f;
     }
     if (p.tinv) {
         for (int i = threadIdx.x; i < r.C * p.tblk; i += blockDim.x) {
@@ -498,12 +498,12 @@ __global__ void __launch_bounds__(256) lift_prefill2_kernel(LiftArgs p) {
         const long long kk = (long long)b0 * p.D + kl;
 #pragma unroll
         for (int t = 0; t < 8; ++t)
-            if (8 * g8 + t < nt) store_u(p.u, p.u_bf16, (long long)(t0 + 8 * g8 + t) * p.K + kk, o[t]);
+            if (8 * g8 + t < nt) store_u(p.u, p.u_bf16, (long long)(t0 + 8 * g8 + t) * p.K + kk, (long long)p.batch * p.K, o[t]);
     }
     if (blockIdx.x == gridDim.x - 1) {  // zero the padded tail of the lifted axis
         const int kreal = nblocks * p.D, npad = p.K - kreal;
         for (int i = threadIdx.x; i < npad * nt; i += blockDim.x)
-            store_u(p.u, p.u_bf16, (long long)(t0 + i / npad) * p.K + kreal + i % npad, 0.f);
+            store_u(p.u, p.u_bf16, (long long)(t0 + i / npad) * p.K + kreal + i % npad, (long long)p.batch * p.K, 0.f);
     }
 }
 
@@ -598,3 +598,5 @@ cudaError_t launch_lift(const void* a, bool a_bf16, int batch, int in, const flo
 }
 
 }  // namespace lq
+
+LQ_DEBUG_FLAG_TAKE(debug_take_lift)

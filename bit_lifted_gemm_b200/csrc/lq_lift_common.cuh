@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "lq_debug.cuh"
+
 namespace lq {
 namespace {
 
@@ -19,7 +21,9 @@ struct LiftArgs {
     int G;   // d-blocks per CTA
 };
 
-__device__ __forceinline__ float load_act(const void* a, int a_bf16, long long idx) {
+// Element idx of an activation buffer of n elements (n bounds the debug build's check).
+__device__ __forceinline__ float load_act(const void* a, int a_bf16, long long idx, long long n) {
+    if (!LQ_IN_BOUNDS(idx, n)) return 0.f;
     if (a_bf16) {
         unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(a) + idx);
         return __uint_as_float((unsigned)h << 16);
@@ -27,7 +31,9 @@ __device__ __forceinline__ float load_act(const void* a, int a_bf16, long long i
     return __ldg(reinterpret_cast<const float*>(a) + idx);
 }
 
-__device__ __forceinline__ void store_u(void* u, int u_bf16, long long idx, float v) {
+// Element idx of u, a buffer of n elements (n bounds the debug build's check).
+__device__ __forceinline__ void store_u(void* u, int u_bf16, long long idx, long long n, float v) {
+    if (!LQ_IN_BOUNDS(idx, n)) return;
     if (u_bf16)
         reinterpret_cast<__nv_bfloat16*>(u)[idx] = __float2bfloat16_rn(v);
     else
@@ -45,7 +51,9 @@ __device__ __forceinline__ void store_u(void* u, int u_bf16, long long idx, floa
 constexpr int WARP_MAXD = 16;
 constexpr int WARP_MAXDD = 64;
 
-__device__ __forceinline__ float4 load_act4(const void* a, int a_bf16, long long idx) {
+// Elements idx .. idx + 3 of an activation buffer of n elements.
+__device__ __forceinline__ float4 load_act4(const void* a, int a_bf16, long long idx, long long n) {
+    if (!LQ_IN_BOUNDS(idx + 3, n)) return make_float4(0.f, 0.f, 0.f, 0.f);
     if (a_bf16) {
         const uint2 h = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const unsigned short*>(a) + idx));
         return make_float4(__uint_as_float(h.x << 16), __uint_as_float(h.x & 0xffff0000u),
@@ -105,13 +113,13 @@ __device__ __forceinline__ void lift_block(const LiftArgs& p, int blk, int lane)
                 for (int q = 0; q < Q; ++q) {
                     const int j4 = lane + 32 * q;
                     const bool ok = t < p.batch && j4 < tb4;
-                    A0[n][q] = ok ? load_act4(p.a, p.a_bf16, arow + ba + 4 * j4) : make_float4(0.f, 0.f, 0.f, 0.f);
-                    A1[n][q] = ok && bb != ba ? load_act4(p.a, p.a_bf16, arow + bb + 4 * j4) : A0[n][q];
+                    A0[n][q] = ok ? load_act4(p.a, p.a_bf16, arow + ba + 4 * j4, (long long)p.batch * p.in) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    A1[n][q] = ok && bb != ba ? load_act4(p.a, p.a_bf16, arow + bb + 4 * j4, (long long)p.batch * p.in) : A0[n][q];
                 }
             } else {
 #pragma unroll
                 for (int i = 0; i < MAXD; ++i)
-                    ap[n][i] = t < p.batch && i < p.d ? load_act(p.a, p.a_bf16, arow + c0 + i) : 0.f;
+                    ap[n][i] = t < p.batch && i < p.d ? load_act(p.a, p.a_bf16, arow + c0 + i, (long long)p.batch * p.in) : 0.f;
             }
         }
         if (Q > 0) {
@@ -142,7 +150,7 @@ __device__ __forceinline__ void lift_block(const LiftArgs& p, int blk, int lane)
                     float acc = 0.f;
 #pragma unroll
                     for (int i = 0; i < MAXD; ++i) acc = fmaf(mc[h][i], ap[n][i], acc);
-                    store_u(p.u, p.u_bf16, (long long)t * p.K + (long long)blk * p.D + j, acc);
+                    store_u(p.u, p.u_bf16, (long long)t * p.K + (long long)blk * p.D + j, (long long)p.batch * p.K, acc);
                 }
             }
         }
@@ -150,7 +158,7 @@ __device__ __forceinline__ void lift_block(const LiftArgs& p, int blk, int lane)
     if (blk == nblocks - 1) {  // zero the padded tail of the lifted axis
         const int kreal = nblocks * p.D;
         for (int t = 0; t < p.batch; ++t)
-            for (int k = kreal + lane; k < p.K; k += 32) store_u(p.u, p.u_bf16, (long long)t * p.K + k, 0.f);
+            for (int k = kreal + lane; k < p.K; k += 32) store_u(p.u, p.u_bf16, (long long)t * p.K + k, (long long)p.batch * p.K, 0.f);
     }
 }
 

@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs
                             v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
                             if (r < p.n1 && tok < p.batch) {
                                 const long long e = (long long)r * p.n2 + 4 * tx;
-                                v[k] = load_act4(p.a, p.a_bf16, (long long)tok * p.in + e);
+                                v[k] = load_act4(p.a, p.a_bf16, (long long)tok * p.in + e, (long long)p.batch * p.in);
                                 if (p.r1) {
                                     const float4 w = __ldg(reinterpret_cast<const float4*>(p.r1 + e));
                                     v[k].x *= w.x;
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs
                 float v = 0.f;
                 if (j2 < p.n2 && tok < p.batch) {
                     const long long e = (long long)r * p.n2 + j2;
-                    v = load_act(p.a, p.a_bf16, (long long)tok * p.in + e);
+                    v = load_act(p.a, p.a_bf16, (long long)tok * p.in + e, (long long)p.batch * p.in);
                     if (p.r1) v *= __ldg(p.r1 + e);
                 }
                 xs[idx] = v;
@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs
 #pragma unroll 4
                     for (int i = 0; i < p.d; ++i) acc = fmaf(ms[i * p.D + lj], yb[i], acc);
                     const float sc = p.r2 ? __ldg(p.r2 + blk0 + b) : 1.f;
-                    store_u(p.u, p.u_bf16, (long long)tok * p.K + (long long)(blk0 + b) * p.D + lj, sc * acc);
+                    store_u(p.u, p.u_bf16, (long long)tok * p.K + (long long)(blk0 + b) * p.D + lj, (long long)p.batch * p.K, sc * acc);
                 }
             }
         }
@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(KR_THREADS, 1) lift_kron_kernel(const KronArgs
             const int k0 = p.in / p.d * p.D, pad = p.K - k0;
             for (int it = tid; it < p.NT * pad; it += KR_THREADS) {
                 const int t = it / pad, k = k0 + (it - t * pad);
-                if (tok0 + t < p.batch) store_u(p.u, p.u_bf16, (long long)(tok0 + t) * p.K + k, 0.f);
+                if (tok0 + t < p.batch) store_u(p.u, p.u_bf16, (long long)(tok0 + t) * p.K + k, (long long)p.batch * p.K, 0.f);
             }
         }
         __syncthreads();  // Y has been read before the next group's X overwrites it
@@ -429,3 +429,5 @@ cudaError_t launch_lift_kron(const void* a, bool a_bf16, int batch, int in, cons
 }
 
 }  // namespace lq
+
+LQ_DEBUG_FLAG_TAKE(debug_take_lift_kron)

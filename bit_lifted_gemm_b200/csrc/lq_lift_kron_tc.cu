@@ -44,6 +44,7 @@
 
 #include <algorithm>
 
+#include "lq_debug.cuh"
 #include "lq_internal.h"
 #include "lq_sm100.cuh"
 
@@ -367,7 +368,7 @@ __global__ void __launch_bounds__(KZ_THREADS, 1)
 template <int DD>
 __device__ __forceinline__ void lift_token(const float* aps, int pitch, int bpr, int bi, int nbi, int nblocks, int e4,
                                            int d, const float (&m)[4][16], const float* r2, __nv_bfloat16* urow,
-                                           int D) {
+                                           int D, int K) {
     constexpr int DL = DD ? DD : 16;
     const int dd = DD ? DD : d;
     int j1 = bi / bpr, off = bi - j1 * bpr;
@@ -393,8 +394,9 @@ __device__ __forceinline__ void lift_token(const float* aps, int pitch, int bpr,
         const float sc = r2 ? __ldg(r2 + b) : 1.f;
         const __nv_bfloat162 h0 = __floats2bfloat162_rn(s4[0] * sc, s4[1] * sc);
         const __nv_bfloat162 h1 = __floats2bfloat162_rn(s4[2] * sc, s4[3] * sc);
-        *reinterpret_cast<uint2*>(urow + (size_t)b * D + 4 * e4) =
-            make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+        if (LQ_IN_BOUNDS((long long)b * D + 4 * e4 + 3, K))  // within the token's row of u
+            *reinterpret_cast<uint2*>(urow + (size_t)b * D + 4 * e4) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
         off += nbi;
         while (off >= bpr) {
             off -= bpr;
@@ -633,18 +635,19 @@ __global__ void __launch_bounds__(KY_THREADS, 1)
             named_barrier_sync(1, 256);  // a' of token k is in shared memory
             const int t = (int)blockIdx.x + k * (int)gridDim.x;
             __nv_bfloat16* urow = p.u + (size_t)t * p.K;
-            if (go && bi < nbi) {
+            const bool row_ok = LQ_IN_BOUNDS(t, p.batch);
+            if (go && row_ok && bi < nbi) {
                 if (p.d == 8)
-                    lift_token<8>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m4, p.r2, urow, p.D);
+                    lift_token<8>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m4, p.r2, urow, p.D, p.K);
                 else if (p.d == 10)
-                    lift_token<10>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m4, p.r2, urow, p.D);
+                    lift_token<10>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m4, p.r2, urow, p.D, p.K);
                 else if (p.d == 16)
-                    lift_token<16>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m4, p.r2, urow, p.D);
+                    lift_token<16>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m4, p.r2, urow, p.D, p.K);
                 else
-                    lift_token<0>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m4, p.r2, urow, p.D);
+                    lift_token<0>(aps, L.pitch, bpr, bi, nbi, nblocks, ec, p.d, m4, p.r2, urow, p.D, p.K);
             }
             // lifted columns past the last block are zero
-            if (go)
+            if (go && row_ok)
                 for (int c = nblocks * p.D + w; c < p.K; c += 256) urow[c] = __float2bfloat16_rn(0.f);
             named_barrier_sync(1, 256);  // every worker is done with a' (and with the snapshot)
             return go;
@@ -806,3 +809,5 @@ cudaError_t launch_lift_kron_tc(const uint16_t* a, int batch, int in, const floa
 }
 
 }  // namespace lq
+
+LQ_DEBUG_FLAG_TAKE(debug_take_lift_kron_tc)

@@ -30,6 +30,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "lq_debug.cuh"
 #include "lq_internal.h"
 #include "lq_sm100.cuh"
 
@@ -130,6 +131,7 @@ __device__ __forceinline__ void lift_chunk(const float* ar, const float* Ms, con
             for (int j = 0; j < W; ++j) acc[j] = fmaf(mr[j], av, acc[j]);
         }
     }
+    if (!LQ_IN_BOUNDS(uidx + W - 1, (long long)p.batch * p.K)) return;
     if (p.u_bf16) {
         __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.u) + uidx;
         if (W == 8) {
@@ -257,6 +259,7 @@ __device__ __forceinline__ void lift_tile_fixed(const float* aps, const float* M
         for (int r = 0; r < 2; ++r) {
             if (r == 1 && !two) break;
             const size_t uo = ui + (r ? rstep : 0);
+            if (!LQ_IN_BOUNDS(uo + W - 1, (long long)p.batch * p.K)) continue;
             if (p.u_bf16) {
                 __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.u) + uo;
                 if (W == 4) {
@@ -483,6 +486,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
                 const int tok = it / tail, e = it - tok * tail;
                 if (t0 + tok >= p.batch) break;
                 const long long idx = (long long)(t0 + tok) * p.K + (long long)nblocks * p.D + e;
+                if (!LQ_IN_BOUNDS(idx, (long long)p.batch * p.K)) continue;
                 if (p.u_bf16)
                     reinterpret_cast<__nv_bfloat16*>(p.u)[idx] = __float2bfloat16_rn(0.f);
                 else
@@ -569,3 +573,5 @@ cudaError_t launch_lift_tc(const uint16_t* a, int batch, int in, const float* ti
 }
 
 }  // namespace lq
+
+LQ_DEBUG_FLAG_TAKE(debug_take_lift_tc)

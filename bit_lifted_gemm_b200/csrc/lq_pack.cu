@@ -5,6 +5,7 @@
 // Both kernels are pure streaming: one thread per packed word, 32 int8 signs
 // moved as two 16-byte vectors. Grids are sized in multiples of the SM count
 // and grid-stride over the words.
+#include "lq_debug.cuh"
 #include "lq_internal.h"
 
 namespace lq {
@@ -29,7 +30,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const int8_t* __restrict__ si
         uint32_t word = 0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) word |= positive_bytes_to_bits(v[i]) << (4 * i);
-        packed[w] = word;
+        if (LQ_IN_BOUNDS(w, nwords)) packed[w] = word;
     }
 }
 
@@ -48,6 +49,7 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint32_t* __restrict_
         uint32_t v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = bits_to_pm1_bytes((word >> (4 * i)) & 0xfu);
+        if (!LQ_IN_BOUNDS(w * 32 + 31, nwords * 32)) continue;
         uint4* dst = reinterpret_cast<uint4*>(signs + w * 32);
         dst[0] = make_uint4(v[0], v[1], v[2], v[3]);
         dst[1] = make_uint4(v[4], v[5], v[6], v[7]);
@@ -78,3 +80,5 @@ cudaError_t launch_unpack(const uint32_t* packed, int out, int K, int8_t* signs,
 }
 
 }  // namespace lq
+
+LQ_DEBUG_FLAG_TAKE(debug_take_pack)

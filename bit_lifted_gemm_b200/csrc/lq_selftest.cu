@@ -3,9 +3,12 @@
 // When the limit passes, the helper latches LQ_DEV_TIMEOUT in the device status
 // word and the kernel returns, so the context stays usable. It exercises the
 // failure-reporting path on the device without faulting or hanging anything.
+// In the debug build a second self-test trips the bounds check once, with no
+// memory access behind it.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "lq_debug.cuh"
 #include "lq_internal.h"
 #include "lq_sm100.cuh"
 
@@ -23,6 +26,11 @@ __global__ void __launch_bounds__(32) wait_timeout_kernel(unsigned* status, unsi
     __syncwarp();
 }
 
+#ifdef LQ_DEBUG
+// Index 1 of an extent of 1: the check fails, latches its flag and no access follows.
+__global__ void bounds_check_kernel() { (void)LQ_IN_BOUNDS(1, 1); }
+#endif
+
 }  // namespace
 
 cudaError_t launch_selftest_wait_timeout(unsigned limit_us, unsigned* status, cudaStream_t st) {
@@ -30,4 +38,16 @@ cudaError_t launch_selftest_wait_timeout(unsigned limit_us, unsigned* status, cu
     return cudaGetLastError();
 }
 
+cudaError_t launch_selftest_bounds(cudaStream_t st) {
+#ifdef LQ_DEBUG
+    bounds_check_kernel<<<1, 1, 0, st>>>();
+    return cudaGetLastError();
+#else
+    (void)st;
+    return cudaErrorNotSupported;
+#endif
+}
+
 }  // namespace lq
+
+LQ_DEBUG_FLAG_TAKE(debug_take_selftest)

@@ -21,8 +21,15 @@
  *  - Argument checks are synchronous and happen before any launch; a call
  *    that fails them launches nothing and returns LQ_ERR_INVALID_ARG.
  *  - A failed launch returns LQ_ERR_CUDA. Errors detected on the device
- *    (a bounded wait that ran out) are latched in a device status word read
- *    by lq_get_device_status().
+ *    (a bounded wait that ran out; in the debug build, an index outside its
+ *    buffer) are latched on the device and read by lq_get_device_status().
+ *  - Debug build: liblq_debug.so, the same entry points compiled with
+ *    -DLQ_DEBUG. Its kernels test the element index of each computed global
+ *    load and store of the pack, lift, Kronecker lift, prefill GEMM and
+ *    encoder kernels against the extent of its buffer (from the call's
+ *    arguments) before the access; a failed test skips the access and latches
+ *    LQ_ERR_BOUNDS. Nothing traps. TMA copies are bounded by their tensor maps
+ *    in both builds. The release library compiles the tests away.
  *  - Packed signs: 32 per uint32, least significant bit first along the
  *    lifted axis, bit 1 = +1, row-major [out][K/32].
  *  - Fault injection for error-path tests (host side only): with the
@@ -54,7 +61,8 @@ typedef enum {
     LQ_ERR_UNSUPPORTED = 2,  /* valid but not supported on this device (needs sm_100) */
     LQ_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
     LQ_ERR_TIMEOUT = 4,      /* a device-side bounded wait expired (from lq_get_device_status) */
-    LQ_ERR_TOO_LARGE = 5     /* the shape needs more scratch than lq_gemv_noalloc's fixed array holds */
+    LQ_ERR_TOO_LARGE = 5,    /* the shape needs more scratch than lq_gemv_noalloc's fixed array holds */
+    LQ_ERR_BOUNDS = 6        /* debug build: a kernel skipped an access outside its buffer (from lq_get_device_status) */
 } lq_status;
 
 typedef enum { LQ_F32 = 0, LQ_BF16 = 1 } lq_dtype;
@@ -88,7 +96,7 @@ LQ_API int lq_unpack_signs(const uint32_t* packed, int out, int K, int8_t* signs
  *                    M_A, M_B the first D-d and last d columns of M;
  *   sign(0) = +1; the smallest ||w - M y||^2 wins, the earliest on ties.
  *   w      : fp32 [rows][in] (the weights to encode, already scaled/whitened)
- *   M      : fp32 [d][D]; 1 <= d <= 16, d <= D <= 63, D - d <= 24, in % d == 0
+ *   M      : fp32 [d][D]; 1 <= d <= 24, d <= D <= 63, D - d <= 24, in % d == 0
  *   packed : uint32 [rows][K/32] (written, the layout lq_gemv reads: block b of
  *            a row occupies bits [b*D, (b+1)*D) of the lifted axis; padding 0)
  *   K      : must equal lq_lifted_dim(in, d, D)
@@ -256,11 +264,24 @@ LQ_API int lq_gemm(const uint32_t* packed, const float* s, int out, int K,
  * sm_100 device (else LQ_ERR_UNSUPPORTED). */
 LQ_API int lq_selftest_wait_timeout(unsigned limit_us, void* stream);
 
+/* Self-test of the debug build's bounds reporting: launches one thread that
+ * tests index 1 against an extent of 1, through the same check the kernels
+ * use, with no memory access behind it. The check fails and latches
+ * LQ_ERR_BOUNDS, which the next lq_get_device_status reports. Returns LQ_OK
+ * after enqueueing it in the debug build, LQ_ERR_UNSUPPORTED in the release
+ * build (whose kernels carry no checks) and on devices other than sm_100. */
+LQ_API int lq_selftest_bounds(void* stream);
+
+/* 1 in the debug build (liblq_debug.so), 0 in the release build. */
+LQ_API int lq_is_debug_build(void);
+
 /* Synchronizes `stream`, then reads and clears, in one atomic exchange on the
  * device, the status word of the stream's device: LQ_OK, or LQ_ERR_TIMEOUT if a
  * kernel there gave up a bounded wait since the last call. A timeout latched
  * meanwhile by a kernel on another stream is either returned or kept for the
- * next call. Returns LQ_ERR_CUDA if a CUDA call fails. */
+ * next call. The debug build also reads and clears the bounds flags of the
+ * device and returns LQ_ERR_BOUNDS, ahead of LQ_ERR_TIMEOUT, if any check
+ * failed since the last call. Returns LQ_ERR_CUDA if a CUDA call fails. */
 LQ_API int lq_get_device_status(void* stream);
 
 #ifdef __cplusplus

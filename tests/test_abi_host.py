@@ -37,7 +37,39 @@ def test_status_strings():
     assert lq.status_str(0) == "LQ_OK"
     assert lq.status_str(1) == "LQ_ERR_INVALID_ARG"
     assert lq.status_str(4) == "LQ_ERR_TIMEOUT"
+    assert lq.status_str(lq.LQ_ERR_BOUNDS) == "LQ_ERR_BOUNDS"
     assert lq.status_str(99) == "LQ_ERR_UNKNOWN"
+
+
+def test_debug_build_exports_and_identifies_itself():
+    """liblq_debug.so, the -DLQ_DEBUG build of the same sources (device-side
+    bounds checks), is built incrementally here, exports every declared symbol
+    and is the library the package loads under LQ_DEBUG=1. The release library
+    says it is not the debug build and refuses the bounds self-test without
+    launching; the debug library, with no GPU, fails its device check."""
+    import importlib.util
+    import subprocess
+    import sys
+
+    import bit_lifted_gemm_b200 as lq
+    spec = importlib.util.spec_from_file_location("lq_build", os.path.join(ROOT, "bit_lifted_gemm_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    path = mod.build(debug=True)
+    assert os.path.basename(path) == "liblq_debug.so"
+    with open(path, "rb") as f:
+        blob = f.read()
+    for name in _declared_symbols():
+        assert name.encode() in blob, name
+    assert lq.lib.lq_is_debug_build() == 0
+    assert lq.lib.lq_selftest_bounds(None) == lq.LQ_ERR_UNSUPPORTED
+    code = ("import bit_lifted_gemm_b200 as lq, os; "
+            "print(lq.lib.lq_is_debug_build(), os.path.basename(lq.LIB_PATH), "
+            "lq.lib.lq_selftest_bounds(None) in (lq.LQ_ERR_CUDA, lq.LQ_ERR_UNSUPPORTED))")
+    env = dict(os.environ, LQ_DEBUG="1")
+    out = subprocess.run([sys.executable, "-c", code], env=env, cwd=ROOT, capture_output=True, text=True,
+                         check=True, timeout=300).stdout.split()
+    assert out == ["1", "liblq_debug.so", "True"]
 
 
 def test_lifted_dim_matches_oracle_closed_form():
@@ -105,7 +137,7 @@ def _c(v):
                                                      10, 24, _c(P), 0, 49152, None]),
     ("kron plan too big (odd n1)", "lq_lift_activations_kron", [_c(P), 0, 1, 16320, None, _c(P), 255, _c(P), 64,
                                                                 None, _c(P), 10, 24, _c(P), 0, 39168, None]),
-    ("encode d > 16", "lq_encode", [_c(P), 4, 340, _c(P), 17, 24, _c(P), 480, None, None]),
+    ("encode d > 24", "lq_encode", [_c(P), 4, 500, _c(P), 25, 32, _c(P), 640, None, None]),
     ("encode D - d > 24", "lq_encode", [_c(P), 4, 40, _c(P), 4, 29, _c(P), 320, None, None]),
     ("encode D < d", "lq_encode", [_c(P), 4, 40, _c(P), 8, 4, _c(P), 32, None, None]),
     ("encode d does not divide in", "lq_encode", [_c(P), 4, 42, _c(P), 4, 12, _c(P), 128, None, None]),

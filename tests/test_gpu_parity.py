@@ -510,7 +510,9 @@ def _block_errors(M, wblocks, y, D):
     (4, 256, 8, 16),   # LQ-16/8
     (2, 30, 6, 14),    # 70 code bits per row: K = 96 with 26 padding bits
     (3, 60, 6, 6),     # D = d: no auxiliary coordinates
-    (2, 96, 16, 20),   # d = 16 (the wide variant), 16 patterns: half the lanes idle
+    (2, 96, 16, 20),   # d = 16, 16 patterns: half the lanes idle
+    (2, 160, 20, 32),  # LQ-32/20 (d = 20, the widest variant): 4096 patterns per block
+    (1, 72, 24, 30),   # d = 24, the largest accepted
 ])
 def test_encode_vs_oracle(lq, rows, in_dim, d, D):
     g = rng_for(62, d * 100 + D, rows)
