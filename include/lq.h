@@ -189,9 +189,15 @@ LQ_API size_t lq_gemv_workspace_size(int out, int K, int batch);
  * signs of its Inf terms.
  * Deterministic. Calls that share a workspace must be
  * ordered (the same stream): overlapping calls race on it. Every pointer must
- * be device memory. The call's first kernel waits for the preceding kernel on
- * the stream before it reads anything. Requires an sm_100 device (else
- * LQ_ERR_UNSUPPORTED). */
+ * be device memory. Launch order: the call's first kernel is a programmatic
+ * dependent of the preceding kernel on the stream. With four or more columns
+ * (and three from 40 MB of packed weights) that first kernel is the quantizer
+ * of u, which waits for the preceding kernel before it reads anything, so no
+ * read of the call can overlap it. With one to three columns on the mma.sync
+ * kernel, packed and s may be read before the preceding kernel completes, when
+ * that kernel lets its dependents start early (this library's lift kernels
+ * do); u is read only after it completes. So the preceding kernel must not
+ * write packed or s. Requires an sm_100 device (else LQ_ERR_UNSUPPORTED). */
 LQ_API int lq_gemv(const uint32_t* packed, const float* s, int out, int K,
             const float* u, int batch, float* o, void* workspace, size_t workspace_bytes, void* stream);
 
