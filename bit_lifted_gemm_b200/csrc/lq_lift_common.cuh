@@ -1,6 +1,7 @@
-// Pieces of the activation lift shared by the lift kernels and the fused
-// lift + GEMV kernel: the argument block, activation / output accessors and the
-// one-warp-per-d-block lift (LiftQuant paper note, "Key designs" 3 and 4).
+// Pieces of the activation lift shared by the block-whitening lift kernels
+// (lq_lift.cu) and the CUDA-core Kronecker lift (lq_lift_kron.cu): the argument
+// block, activation / output accessors (bounds-checked in the debug build) and
+// the one-warp-per-d-block lift (LiftQuant paper note, "Key designs" 3 and 4).
 #pragma once
 
 #include <cuda_bf16.h>

@@ -147,13 +147,24 @@ LQ_API int lq_lift_activations(const void* a, int a_dtype, int batch, int in,
  *   M, d, D, u, u_dtype, K : as lq_lift_activations (in % d == 0)
  * Kronecker entry ((i1, i2), (j1, j2)) is q1[i1][j1] * q2[i2][j2] with channel
  * i = i1 * n2 + i2, so for one token, X = a reshaped row-major to n1 x n2,
- * (Q1 kron Q2) x = Q1 X Q2^T: in * (n1 + n2) multiply-adds, fp32 throughout.
- * Computed as (Q1 X) Q2^T with each CTA owning a slice of rows of the result,
- * so no scratch memory and no exchange between CTAs; shapes whose
- * shared-memory plan does not fit (e.g. a large odd n1) return
- * LQ_ERR_INVALID_ARG. Launched as a programmatic dependent of the preceding
- * kernel; it reads a only after that kernel completes. Requires an sm_100
- * device (else LQ_ERR_UNSUPPORTED). */
+ * (Q1 kron Q2) x = Q1 X Q2^T: in * (n1 + n2) multiply-adds per token.
+ * Two implementations, chosen by shape:
+ *  - Prefill on the tensor cores: bf16 a and u, batch >= 64, 8 <= n1 <= 64,
+ *    16 <= n2 <= 128 a multiple of 16, d <= 16 dividing n2, D >= 2 d a
+ *    multiple of 4. Z = (r1 o X) Q2^T over all tokens, then Q1 Z per token,
+ *    with the fp32 factors and Z split into three bf16 parts (24 significant
+ *    bits, fp32 accumulation: the accuracy class of fp32 arithmetic), then
+ *    the lift on the CUDA cores. Z of token t is kept in row t of u until the
+ *    lift of t overwrites it, so u must not alias a. Bounded waits inside
+ *    report LQ_ERR_TIMEOUT through lq_get_device_status.
+ *  - Otherwise (decode batches, fp32 a or u, other factor sizes): fp32
+ *    throughout, computed as (Q1 X) Q2^T with each CTA owning a slice of rows
+ *    of the result, no scratch memory and no exchange between CTAs; shapes
+ *    whose shared-memory plan does not fit (e.g. a large odd n1) return
+ *    LQ_ERR_INVALID_ARG.
+ * Launched as a programmatic dependent of the preceding kernel; it reads a
+ * only after that kernel completes. Requires an sm_100 device (else
+ * LQ_ERR_UNSUPPORTED). */
 LQ_API int lq_lift_activations_kron(const void* a, int a_dtype, int batch, int in,
                                     const float* r1, const float* q1, int n1, const float* q2, int n2,
                                     const float* r2, const float* M, int d, int D,
