@@ -185,6 +185,20 @@ def test_fault_injection_launch(monkeypatch):
     assert lq.lib.lq_gemv(_c(P), _c(P), 8, 64, _c(P), 0, _c(P), _c(W), BIG, None) == lq.LQ_ERR_INVALID_ARG
 
 
+def test_encode_accepts_every_tabulated_code(monkeypatch):
+    """The encoder's argument checks accept every LQ-D/d code of the pages' table,
+    LQ-32/20 (d = 20) included, and d up to 24; with LQ_FAULT=launch an accepted
+    call returns LQ_ERR_CUDA right after its checks, without launching."""
+    import bit_lifted_gemm_b200 as lq
+    monkeypatch.setenv("LQ_FAULT", "launch")
+    for d, D in ((20, 32), (16, 32), (8, 16), (14, 30), (10, 24), (24, 48)):
+        in_dim = d * 8
+        K = lq.lifted_dim(in_dim, d, D)
+        assert lq.lib.lq_encode(_c(P), 2, in_dim, _c(P), d, D, _c(P), K, None, None) == lq.LQ_ERR_CUDA, (d, D)
+    assert lq.lib.lq_encode(_c(P), 2, 200, _c(P), 25, 40, _c(P), lq.lifted_dim(200, 25, 40), None,
+                            None) == lq.LQ_ERR_INVALID_ARG
+
+
 def test_gemv_rejects_rows_beyond_the_plan():
     """Row lengths that are not a multiple of four words run on the mma.sync
     kernel, whose CTAs keep 64-bit partial sums for their rows in shared memory;
