@@ -516,7 +516,11 @@ def bench_prefill(torch, lq, name, tokens, reps=10):
 
 GRAPH_STEPS = 1024      # steps per CUDA graph of the timed region
 GEMV_LAUNCHES = 2048    # GEMV-alone launches behind the roofline, whatever --steps is
-LAUNCHES_PER_STEP = 3   # lift, u quantizer, GEMV contraction
+# Kernels of this library per timed step: the lift and the GEMV. At one column the
+# GEMV is the mma.sync kernel, which quantizes u inside its CTAs and covers K in one
+# launch for every decode layer timed here (the ncu launch list of the step shows
+# the two); the row-sharded mode runs the same two per rank plus an NCCL all-gather.
+LAUNCHES_PER_STEP = 2
 
 
 def spawn_ranks(args):
