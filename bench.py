@@ -734,8 +734,11 @@ def main():
         import oracle
         nthreads = oracle.threads_available()
         v, dt, desc = oracle_sample(args.workload, 15.0, nthreads)
+        v1, dt1, desc1 = oracle_sample(args.workload, 4.0, 1)
         result["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": nthreads, "kind": "oracle",
-                                  "sample": desc + f" ({dt:.1f} s)"}
+                                  "sample": desc + f" ({dt:.1f} s)",
+                                  "single_thread": {"value": v1, "unit": "GB/s", "cores": 1,
+                                                    "sample": desc1 + f" ({dt1:.1f} s)"}}
 
     assert lq.get_device_status() == lq.LQ_OK
     if rank == 0:
