@@ -86,6 +86,31 @@ bool all_device(std::initializer_list<const void*> ps) {
     return true;
 }
 
+// A byte range [p, p + n) that a call reads, or writes.
+struct Span {
+    const void* p;
+    size_t n;
+    bool written;
+};
+
+// True when a range the call writes shares a byte with another of its ranges:
+// an output aliasing an input (or another output) would be read and written by
+// different CTAs in no fixed order. Null pointers and empty ranges never overlap;
+// sizes come from validated int arguments, so the sums cannot wrap.
+bool aliased(std::initializer_list<Span> spans) {
+    const Span* v = spans.begin();
+    const size_t n = spans.size();
+    for (size_t i = 0; i < n; ++i)
+        for (size_t j = i + 1; j < n; ++j) {
+            if (!(v[i].written || v[j].written) || !v[i].p || !v[j].p || !v[i].n || !v[j].n) continue;
+            const uintptr_t a = reinterpret_cast<uintptr_t>(v[i].p), b = reinterpret_cast<uintptr_t>(v[j].p);
+            if (a < b + v[j].n && b < a + v[i].n) return true;
+        }
+    return false;
+}
+
+size_t nbytes(long long count, size_t elem) { return (size_t)count * elem; }
+
 // Device address of the status word on the current device (looked up once per device).
 unsigned* status_word(int* err) {
     static unsigned* addr[kMaxDevices] = {};
@@ -149,6 +174,8 @@ int lq_lifted_dim(int in, int d, int D) {
 int lq_pack_signs(const int8_t* signs_pm1, int out, int K, uint32_t* packed, void* stream) {
     if (!signs_pm1 || !packed || !aligned16(signs_pm1) || !aligned16(packed)) return LQ_ERR_INVALID_ARG;
     if (out < 1 || K < 32 || K % 32 != 0) return LQ_ERR_INVALID_ARG;
+    if (aliased({{signs_pm1, nbytes((long long)out * K, 1), false}, {packed, nbytes((long long)out * (K / 32), 4), true}}))
+        return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     if (!all_device({signs_pm1, packed})) return LQ_ERR_INVALID_ARG;
     return from_cuda(lq::launch_pack(signs_pm1, out, K, packed, static_cast<cudaStream_t>(stream)));
@@ -157,6 +184,8 @@ int lq_pack_signs(const int8_t* signs_pm1, int out, int K, uint32_t* packed, voi
 int lq_unpack_signs(const uint32_t* packed, int out, int K, int8_t* signs_pm1, void* stream) {
     if (!signs_pm1 || !packed || !aligned16(signs_pm1) || !aligned16(packed)) return LQ_ERR_INVALID_ARG;
     if (out < 1 || K < 32 || K % 32 != 0) return LQ_ERR_INVALID_ARG;
+    if (aliased({{packed, nbytes((long long)out * (K / 32), 4), false}, {signs_pm1, nbytes((long long)out * K, 1), true}}))
+        return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     if (!all_device({packed, signs_pm1})) return LQ_ERR_INVALID_ARG;
     return from_cuda(lq::launch_unpack(packed, out, K, signs_pm1, static_cast<cudaStream_t>(stream)));
@@ -171,6 +200,11 @@ int lq_lift_activations(const void* a, int a_dtype, int batch, int in, const flo
     if (batch < 1 || in < 1 || d < 1 || d > 64 || D < 1 || D > 256 || d * D > 4096) return LQ_ERR_INVALID_ARG;
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
     if (tinv && (tblk < 1 || tblk > 256 || in % tblk != 0)) return LQ_ERR_INVALID_ARG;
+    if (aliased({{a, nbytes((long long)batch * in, a_dtype == LQ_BF16 ? 2 : 4), false},
+                 {tinv, tinv ? nbytes((long long)in * tblk, 4) : 0, false},
+                 {M, nbytes((long long)d * D, 4), false},
+                 {u, nbytes((long long)batch * K, u_dtype == LQ_BF16 ? 2 : 4), true}}))
+        return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
@@ -197,6 +231,14 @@ int lq_lift_activations_kron(const void* a, int a_dtype, int batch, int in, cons
     if (n1 < 1 || n1 > 256 || n2 < 1 || n2 > 128 || n1 * n2 != in || in % d != 0) return LQ_ERR_INVALID_ARG;
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
     if (!lq::lift_kron_supported(batch, in, n1, n2, d, D)) return LQ_ERR_INVALID_ARG;
+    if (aliased({{a, nbytes((long long)batch * in, a_dtype == LQ_BF16 ? 2 : 4), false},
+                 {r1, nbytes(in, 4), false},
+                 {q1, nbytes((long long)n1 * n1, 4), false},
+                 {q2, nbytes((long long)n2 * n2, 4), false},
+                 {r2, nbytes(in / d, 4), false},
+                 {M, nbytes((long long)d * D, 4), false},
+                 {u, nbytes((long long)batch * K, u_dtype == LQ_BF16 ? 2 : 4), true}}))
+        return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
@@ -221,6 +263,11 @@ int lq_encode(const float* w, int rows, int in, const float* M, int d, int D, ui
     if (rows < 1 || in < 1 || d < 1 || d > 24 || D < d || D > 63 || D - d > 24 || in % d != 0)
         return LQ_ERR_INVALID_ARG;
     if (lq_lifted_dim(in, d, D) != K) return LQ_ERR_INVALID_ARG;
+    if (aliased({{w, nbytes((long long)rows * in, 4), false},
+                 {M, nbytes((long long)d * D, 4), false},
+                 {packed, nbytes((long long)rows * (K / 32), 4), true},
+                 {err, err ? nbytes((long long)rows * (in / d), 4) : 0, true}}))
+        return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
@@ -254,6 +301,12 @@ int lq_gemv(const uint32_t* packed, const float* s, int out, int K, const float*
     if (out < 1 || K < 32 || K % 32 != 0 || batch < 1 || batch > 16) return LQ_ERR_INVALID_ARG;
     const size_t need = lq::gemv_workspace_size(out, K, batch);
     if (need == 0 || workspace_bytes < need) return LQ_ERR_INVALID_ARG;
+    if (aliased({{packed, nbytes((long long)out * (K / 32), 4), false},
+                 {s, nbytes(out, 4), false},
+                 {u, nbytes((long long)batch * K, 4), false},
+                 {o, nbytes((long long)batch * out, 4), true},
+                 {workspace, need, true}}))
+        return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
@@ -282,6 +335,15 @@ int lq_lift_gemv(const void* a, int a_dtype, int batch, int in, const float* tin
     if (out < 1) return LQ_ERR_INVALID_ARG;
     const size_t need = lq::gemv_workspace_size(out, K, batch);
     if (need == 0 || workspace_bytes < need) return LQ_ERR_INVALID_ARG;
+    if (aliased({{a, nbytes((long long)batch * in, a_dtype == LQ_BF16 ? 2 : 4), false},
+                 {tinv, tinv ? nbytes((long long)in * tblk, 4) : 0, false},
+                 {M, nbytes((long long)d * D, 4), false},
+                 {packed, nbytes((long long)out * (K / 32), 4), false},
+                 {s, nbytes(out, 4), false},
+                 {u, nbytes((long long)batch * K, 4), true},
+                 {o, nbytes((long long)batch * out, 4), true},
+                 {workspace, need, true}}))
+        return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
@@ -299,6 +361,11 @@ int lq_gemm(const uint32_t* packed, const float* s, int out, int K, const uint16
     if (!packed || !s || !u_bf16 || !o) return LQ_ERR_INVALID_ARG;
     if (!aligned16(packed) || !aligned16(s) || !aligned16(u_bf16) || !aligned16(o)) return LQ_ERR_INVALID_ARG;
     if (out < 1 || K < 32 || K % 32 != 0 || tokens < 1) return LQ_ERR_INVALID_ARG;
+    if (aliased({{packed, nbytes((long long)out * (K / 32), 4), false},
+                 {s, nbytes(out, 4), false},
+                 {u_bf16, nbytes((long long)tokens * K, 2), false},
+                 {o, nbytes((long long)tokens * out, 4), true}}))
+        return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;
@@ -397,6 +464,11 @@ int lq_gemv_noalloc(const uint32_t* packed, const float* s, int out, int K, cons
     const size_t need = lq::gemv_workspace_size(out, K, batch);
     if (need == 0) return LQ_ERR_INVALID_ARG;
     if (need > LQ_GEMV_NOALLOC_SCRATCH_BYTES) return LQ_ERR_TOO_LARGE;
+    if (aliased({{packed, nbytes((long long)out * (K / 32), 4), false},
+                 {s, nbytes(out, 4), false},
+                 {u, nbytes((long long)batch * K, 4), false},
+                 {o, nbytes((long long)batch * out, 4), true}}))
+        return LQ_ERR_INVALID_ARG;
     if (fault_is("launch")) return LQ_ERR_CUDA;
     const int sm = is_sm100();
     if (sm < 0) return LQ_ERR_CUDA;

@@ -20,6 +20,10 @@
  *    stream-ordered and asynchronous: they return after enqueueing work.
  *  - Argument checks are synchronous and happen before any launch; a call
  *    that fails them launches nothing and returns LQ_ERR_INVALID_ARG.
+ *  - No output may share a byte with an input or another output of the same
+ *    call (in-place calls are refused): the checks compare the byte ranges
+ *    that the pointers and the sizes in the arguments imply (for a workspace,
+ *    the bytes the shape needs). Inputs may overlap one another.
  *  - A failed launch returns LQ_ERR_CUDA. Errors detected on the device
  *    (a bounded wait that ran out; in the debug build, an index outside its
  *    buffer) are latched on the device and read by lq_get_device_status().

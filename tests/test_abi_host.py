@@ -89,6 +89,13 @@ def _c(v):
     return ctypes.c_void_p(v)
 
 
+def _far(i):
+    """Distinct fake buffer addresses, 64 GiB apart: never dereferenced (the calls
+    that get them return before any launch), far enough apart that no range of
+    any tested shape reaches the next."""
+    return _c((i + 1) << 36)
+
+
 @pytest.mark.parametrize("case", [
     ("pack null", "lq_pack_signs", [None, 4, 32, _c(P), None]),
     ("pack K%32", "lq_pack_signs", [_c(P), 4, 48, _c(P), None]),
@@ -178,10 +185,10 @@ def test_fault_injection_launch(monkeypatch):
     pointers; argument checks still come first."""
     import bit_lifted_gemm_b200 as lq
     monkeypatch.setenv("LQ_FAULT", "launch")
-    assert lq.lib.lq_pack_signs(_c(P), 4, 32, _c(P), None) == lq.LQ_ERR_CUDA
-    assert lq.lib.lq_gemv(_c(P), _c(P), 8, 64, _c(P), 1, _c(P), _c(W), BIG, None) == lq.LQ_ERR_CUDA
-    assert lq.lib.lq_gemm(_c(P), _c(P), 8, 64, _c(P), 4, _c(P), None) == lq.LQ_ERR_CUDA
-    assert lq.lib.lq_encode(_c(P), 4, 40, _c(P), 4, 12, _c(P), 128, None, None) == lq.LQ_ERR_CUDA
+    assert lq.lib.lq_pack_signs(_far(0), 4, 32, _far(1), None) == lq.LQ_ERR_CUDA
+    assert lq.lib.lq_gemv(_far(0), _far(1), 8, 64, _far(2), 1, _far(3), _far(4), BIG, None) == lq.LQ_ERR_CUDA
+    assert lq.lib.lq_gemm(_far(0), _far(1), 8, 64, _far(2), 4, _far(3), None) == lq.LQ_ERR_CUDA
+    assert lq.lib.lq_encode(_far(0), 4, 40, _far(1), 4, 12, _far(2), 128, None, None) == lq.LQ_ERR_CUDA
     assert lq.lib.lq_gemv(_c(P), _c(P), 8, 64, _c(P), 0, _c(P), _c(W), BIG, None) == lq.LQ_ERR_INVALID_ARG
 
 
@@ -194,7 +201,7 @@ def test_encode_accepts_every_tabulated_code(monkeypatch):
     for d, D in ((20, 32), (16, 32), (8, 16), (14, 30), (10, 24), (24, 48)):
         in_dim = d * 8
         K = lq.lifted_dim(in_dim, d, D)
-        assert lq.lib.lq_encode(_c(P), 2, in_dim, _c(P), d, D, _c(P), K, None, None) == lq.LQ_ERR_CUDA, (d, D)
+        assert lq.lib.lq_encode(_far(0), 2, in_dim, _far(1), d, D, _far(2), K, None, None) == lq.LQ_ERR_CUDA, (d, D)
     assert lq.lib.lq_encode(_c(P), 2, 200, _c(P), 25, 40, _c(P), lq.lifted_dim(200, 25, 40), None,
                             None) == lq.LQ_ERR_INVALID_ARG
 
@@ -226,8 +233,57 @@ def test_gemv_plan_fits_every_configured_layer(monkeypatch):
         for batch in (1, 2, 4, 8, 16):
             ws = lq.gemv_workspace_size(cfg.out, cfg.K, batch)
             assert ws > 0, (cfg.name, batch)
-            rc = lq.lib.lq_gemv(_c(P), _c(P), cfg.out, cfg.K, _c(P), batch, _c(P), _c(W), ws, None)
+            rc = lq.lib.lq_gemv(_far(0), _far(1), cfg.out, cfg.K, _far(2), batch, _far(3), _far(4), ws, None)
             assert rc == lq.LQ_ERR_CUDA, (cfg.name, batch)
             # one byte short of the workspace the plan needs is refused
             rc = lq.lib.lq_gemv(_c(P), _c(P), cfg.out, cfg.K, _c(P), batch, _c(P), _c(W), ws - 1, None)
             assert rc == lq.LQ_ERR_INVALID_ARG, (cfg.name, batch)
+
+
+def test_outputs_may_not_overlap_other_buffers(monkeypatch):
+    """Every entry point refuses, before any launch, an output range that shares a
+    byte with an input or another output of the same call (sizes from the
+    arguments); ranges that merely touch are fine, and inputs may share memory.
+    LQ_FAULT=launch makes accepted calls return LQ_ERR_CUDA right after the
+    checks, so no fake pointer is ever dereferenced."""
+    import bit_lifted_gemm_b200 as lq
+    monkeypatch.setenv("LQ_FAULT", "launch")
+    base = 1 << 36
+    INV, OK = lq.LQ_ERR_INVALID_ARG, lq.LQ_ERR_CUDA
+    # pack: signs 4 x 32 bytes, packed 4 x 1 words = 16 bytes
+    assert lq.lib.lq_pack_signs(_c(base), 4, 32, _c(base + 128), None) == OK       # packed right after signs
+    assert lq.lib.lq_pack_signs(_c(base), 4, 32, _c(base + 112), None) == INV      # last 16 bytes of signs
+    assert lq.lib.lq_unpack_signs(_c(base), 4, 32, _c(base + 16), None) == OK
+    assert lq.lib.lq_unpack_signs(_c(base + 16), 4, 32, _c(base), None) == INV     # signs cover packed
+    # lift: a fp32 [2][640] = 5120 B, M 10 x 24 fp32, u fp32 [2][1536] = 12288 B
+    lift = lambda a, M, u: lq.lib.lq_lift_activations(_c(a), 0, 2, 640, None, 0, _c(M), 10, 24, _c(u), 0, 1536, None)
+    assert lift(base, 2 * base, base + 5120) == OK
+    assert lift(base, 2 * base, base) == INV                                      # in place
+    assert lift(base, base + 5120, 2 * base) == OK                                # inputs adjacent
+    assert lift(base, 2 * base, 2 * base + 944) == INV                            # u covers the end of M (960 B)
+    # Kronecker lift: u over q2
+    kron = lambda u: lq.lib.lq_lift_activations_kron(_c(base), 0, 1, 640, None, _c(2 * base), 8, _c(3 * base), 80,
+                                                      None, _c(4 * base), 10, 24, _c(u), 0, 1536, None)
+    assert kron(5 * base) == OK
+    assert kron(3 * base + 16) == INV
+    # GEMV: o [1][8] fp32 against u [1][64]; the workspace range is what the plan needs
+    ws = lq.gemv_workspace_size(8, 64, 1)
+    gemv = lambda o, w: lq.lib.lq_gemv(_c(base), _c(2 * base), 8, 64, _c(3 * base), 1, _c(o), _c(w), BIG, None)
+    assert gemv(4 * base, 5 * base) == OK
+    assert gemv(3 * base + 224, 5 * base) == INV                                  # o over the end of u (256 B)
+    assert gemv(4 * base, 4 * base + 16) == INV                                   # workspace over o
+    assert gemv(4 * base, 4 * base + 256) == OK                                   # workspace right after o (32 B)
+    assert lq.lib.lq_gemv_noalloc(_c(base), _c(2 * base), 8, 64, _c(3 * base), 1, _c(base), None) == INV
+    # lift + GEMV: u over a, o over the workspace
+    lg = lambda u, o, w: lq.lib.lq_lift_gemv(_c(base), 0, 1, 640, None, 0, _c(2 * base), 10, 24, _c(3 * base),
+                                              _c(4 * base), 8, 1536, _c(u), _c(o), _c(w), BIG, None)
+    assert lg(5 * base, 6 * base, 7 * base) == OK
+    assert lg(base + 1024, 6 * base, 7 * base) == INV
+    assert lg(5 * base, 7 * base, 7 * base) == INV
+    # GEMM: o over the packed signs; encode: err over packed
+    assert lq.lib.lq_gemm(_c(base), _c(2 * base), 8, 64, _c(3 * base), 4, _c(4 * base), None) == OK
+    assert lq.lib.lq_gemm(_c(base), _c(2 * base), 8, 64, _c(3 * base), 4, _c(base), None) == INV
+    enc = lambda packed, err: lq.lib.lq_encode(_c(base), 4, 40, _c(2 * base), 4, 12, _c(packed), 128, _c(err), None)
+    assert enc(3 * base, 4 * base) == OK
+    assert enc(3 * base, 3 * base + 48) == INV                                    # packed is 4 x 16 bytes
+    assert enc(3 * base, 3 * base + 64) == OK
