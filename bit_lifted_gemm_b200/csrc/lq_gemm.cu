@@ -61,7 +61,6 @@ struct TileTA {
     static_assert(A_COL + S * A_COLS <= 512, "accumulators and A stages exceed tensor memory");
 };
 constexpr int TA_ISSUERS = 2, TA_STAGES = 4;
-constexpr bool TA_EAGER = false, TA_SPLIT = true;
 
 // Expand 16 sign bits (bit i = element i of a k-run) into 8 bf16x2 words:
 // word i holds elements (2i, 2i+1) as +1.0 (0x3F80) or -1.0 (0xBF80).
@@ -490,12 +489,6 @@ __global__ void __launch_bounds__(TileTA<BN, NI, S>::THREADS, 1)
                 // word j holds k-elements (2j, 2j+1): TMEM column j of the stage
                 tmem_st_32x32b_x32(a_lane + st * A_COLS, v);
                 pending = st;
-                if (TA_EAGER) {
-                    tmem_st_wait();
-                    tc_fence_before();
-                    mbar_arrive(full0 + 8 * st);
-                    pending = -1;
-                }
             }
 #pragma unroll
             for (int q = 0; q < 16; ++q) cur[q] = nxt[q];
@@ -588,7 +581,7 @@ cudaError_t launch_tile(const uint32_t* packed, const float* s, int out, int K, 
     }
     dim3 grid((out + BM - 1) / BM, (tokens + BN - 1) / BN, 1);
     const int nkb = (K + BK - 1) / BK;
-    if ((!kTA || TA_SPLIT) && (long long)grid.x * grid.y < num_sms && nkb >= 16) {  // too few tiles for the SMs: split K in two
+    if ((long long)grid.x * grid.y < num_sms && nkb >= 16) {  // too few tiles for the SMs: split K in two
         grid.z = 2;
         cudaError_t e = cudaMemsetAsync(o, 0, (size_t)tokens * out * sizeof(float), st);
         if (e != cudaSuccess) return e;
