@@ -422,3 +422,35 @@ def test_encode_search_square_closed_form():
     x = np.linalg.solve(M, w.T).T
     want = ((x >= 0).astype(np.uint64) << np.arange(d, dtype=np.uint64)[None, :]).sum(axis=1)
     assert np.array_equal(y, want.astype(np.uint64))
+
+
+# ---------------------------------------------------------------- Gaussian source
+
+def test_gaussian_table_info_and_rate_distortion():
+    """The note's Gaussian-source table: Info is -1/2 log2 MSE on every row (to the
+    printed rounding), and no code beats the rate-distortion bound of an i.i.d.
+    N(0, 1) source at its D/d bits per weight, MSE >= 2^(-2 D/d)."""
+    rows = _golden_lines("gaussian_source.txt")
+    assert len(rows) == 5
+    for D, d, bits, mse, info in rows:
+        D, d, bits, mse, info = int(D), int(d), float(bits), float(mse), float(info)
+        assert abs(bits - D / d) <= 0.005
+        assert abs(info - (-0.5 * np.log2(mse))) <= 0.015, (D, d)
+        assert mse >= 2.0 ** (-2.0 * D / d), (D, d)
+
+
+@pytest.mark.parametrize("d,D", [(8, 16), (10, 24), (6, 14)])
+def test_encode_gaussian_source_above_rate_distortion(d, D):
+    """The search on i.i.d. N(0, 1) weights with M ~ N(0, 1/D): its per-weight
+    squared error, computed independently here from the returned patterns, equals
+    the oracle's and stays above 2^(-2 D/d), which no quantizer at D/d bits per
+    weight can beat on this source."""
+    g = rng_for(92, d, D)
+    M = g.standard_normal((d, D)) / np.sqrt(D)
+    w = g.standard_normal((300, d))
+    y, e = oracle.encode_blocks(M, w, nthreads=4)
+    s = oracle.patterns_to_signs(y, D).astype(np.float64)
+    e_np = np.sum((w - s @ M.T) ** 2, axis=1)
+    assert np.allclose(e, e_np, rtol=1e-12, atol=1e-14)
+    mse = float(np.mean(e_np)) / d
+    assert mse >= 2.0 ** (-2.0 * D / d), mse
